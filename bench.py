@@ -1,0 +1,427 @@
+"""Benchmark: HiLS forward prefill (TFLOP/s) and paged decode (tok/s) on B200.
+
+One step = one full prefill forward pass (summaries, scores + Top-K,
+selected-chunk and own-chunk attention, fusion) of the 345M-shaped workload:
+batch 4, 16 heads, N = 8192, d = 64, B = 64, Top-K = 16, bf16 inputs with
+planted needles.  `value` is whole-job TFLOP/s of algorithmic FLOPs
+(4*d*(K_eff*B + own keys) per query head, the selected-chunk and own-chunk
+QK^T + PV work), device-timed with CUDA events, inputs resident in HBM, L2
+flushed (256 MB write) between steps outside the timed events.
+
+Decode is reported beside it (tok/s at 32K/128K/512K, CUDA-graph replay).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs an independent replica (no collective on
+the data path); rank 0 prints one JSON line with the max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from hils_inputs import CONFIGS, decode_inputs, prefill_inputs  # noqa: E402
+
+PREFILL = CONFIGS["prefill_345m"]
+METRIC = "HiLS fwd prefill TFLOP/s + decode tok/s; % of roofline on 1 B200"
+
+
+def algorithmic_flops(batch, heads_q, seq_len, head_dim, top_k, chunk=64):
+    i = np.arange(seq_len)
+    keff = np.minimum(top_k, i // chunk)
+    keys = keff * chunk + (i % chunk) + 1
+    return float(4 * head_dim * keys.sum() * batch * heads_q)
+
+
+def decode_bytes(cfg):
+    b, h, g, d, K = cfg["batch"], cfg["heads_q"], cfg["heads_kv"], cfg["head_dim"], cfg["top_k"]
+    L = cfg["seq_len"]
+    own = (L - 1) // 64
+    keff = min(K, own)
+    own_keys = L - own * 64
+    kv = b * g * (keff * 64 + own_keys) * d * 2 * 2
+    summ = b * own * h * (d + 1) * 4
+    qo = b * h * d * 2 * 2
+    return float(kv + summ + qo), float(kv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    Q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------- CPU baseline (oracle)
+def cpu_baseline(seconds_budget=20.0):
+    """Times the fp64 oracle on a bounded sample of the prefill workload."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import hils_oracle as O
+    cfg = dict(PREFILL)
+    inp = prefill_inputs(seed=0, device="cpu", **cfg)
+    n = cfg["seq_len"]
+    # sample: whole (batch, head) pairs in order until the time budget is spent
+    t0 = time.perf_counter()
+    flops, done_rows, pairs = 0.0, 0, 0
+    rows = np.arange(n)
+    keff = np.minimum(cfg["top_k"], rows // 64)
+    pair_flops = float(4 * cfg["head_dim"] * (keff * 64 + rows % 64 + 1).sum())
+    with threadpool_limits(limits=1):
+        for bi in range(cfg["batch"]):
+            for hi in range(cfg["heads_q"]):
+                if time.perf_counter() - t0 >= seconds_budget:
+                    break
+                O.forward(inp.q[bi:bi + 1, hi:hi + 1], inp.k[bi:bi + 1, hi:hi + 1],
+                          inp.v[bi:bi + 1, hi:hi + 1], inp.landmark[bi:bi + 1, hi:hi + 1], 64,
+                          cfg["top_k"])
+                flops += pair_flops
+                pairs += 1
+    dt = time.perf_counter() - t0
+    done = pairs * n
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"{pairs} of {cfg['batch'] * cfg['heads_q']} (batch, head) pairs, all {n} query rows "
+                      f"each (summaries, scores, Top-K, attention, fusion), {dt:.1f} s, fp64 numpy, "
+                      f"BLAS limited to 1 thread"}
+
+
+# ---------------------------------------------------------------------------- prefill (ours)
+def run_prefill(args, ws_world, rank, local):
+    import chunk_wise_hierarchical_b200 as hils
+    dev = torch.device("cuda", local)
+    cfg = PREFILL
+    inp = prefill_inputs(seed=rank, device=dev, **cfg)
+    q, k, v, lm = inp.q, inp.k, inp.v, inp.landmark
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    K = cfg["top_k"]
+    out = torch.empty_like(q)
+    sh = hils.make_shape(b, h, g, d, n, K, 1)
+    C = n // 64
+    kbar = torch.empty((b, h, C, d), dtype=torch.float32, device=dev)
+    hb = torch.empty((b, h, C), dtype=torch.float32, device=dev)
+    idx = torch.empty((b, g, n, K), dtype=torch.int32, device=dev)
+    ssel = torch.empty((b, h, n, K), dtype=torch.float32, device=dev)
+    ws_sel = hils.new_workspace(sh, hils.OP_ATTEND_SELECTED, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    flops = algorithmic_flops(b, h, n, d, K)
+
+    def step(evs=None):
+        # the three stages of hils_attend, called separately so the attention kernel can be timed
+        if evs: evs[0].record(stream)
+        kb, hbb = kbar, hb
+        lib = hils.lib()
+        import ctypes
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        st = ctypes.c_void_p(stream.cuda_stream)
+        r = lib.hils_summarize(ctypes.byref(sh), P(k), P(lm), P(kb), P(hbb), st)
+        if evs: evs[1].record(stream)
+        r |= lib.hils_select(ctypes.byref(sh), P(q), P(kb), P(hbb), P(idx), P(ssel), None, 0, st)
+        if evs: evs[2].record(stream)
+        r |= lib.hils_attend_selected(ctypes.byref(sh), P(q), P(k), P(v), P(idx), P(ssel), P(out),
+                                      P(ws_sel), ws_sel.numel(), st)
+        if evs: evs[3].record(stream)
+        if r != 0:
+            raise RuntimeError(f"HiLS call failed: {r}")
+
+    for _ in range(args.warmup):
+        step()
+    barrier(ws_world)
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with Clocks(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evsets[i])
+        barrier(ws_world)
+    tot = [e[0].elapsed_time(e[3]) for e in evsets]
+    att = [e[2].elapsed_time(e[3]) for e in evsets]
+    summ = [e[0].elapsed_time(e[1]) for e in evsets]
+    sel = [e[1].elapsed_time(e[2]) for e in evsets]
+    ms_step = max_over_ranks(sum(tot) / len(tot), ws_world)
+    ms_att = sum(att) / len(att)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    host = [t.cpu().pin_memory() for t in (q, k, v, lm)]
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    call = hils.Prefill(b, h, g, n, d, K, torch.bfloat16, device=dev)
+    dq, dk, dv, dl = (torch.empty_like(t) for t in (q, k, v, lm))
+    dout = torch.empty_like(q)
+
+    def e2e_step():
+        for dst, src in zip((dq, dk, dv, dl), host):
+            dst.copy_(src, non_blocking=True)
+        call(dq, dk, dv, dl, out=dout)
+        host_out.copy_(dout, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    n_e2e = max(2, args.steps // 2)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, ws_world)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = host_out.numel() * host_out.element_size()
+    return dict(flops=flops, ms_step=ms_step, ms_att=ms_att, ms_summ=sum(summ) / len(summ),
+                ms_sel=sum(sel) / len(sel), ms_e2e=ms_e2e, h2d=h2d, d2h=d2h, clocks=clk.summary(),
+                launches_per_step=3)
+
+
+# ---------------------------------------------------------------------------- decode (ours)
+def run_decode(name, n_caches, dev, reps=50):
+    import chunk_wise_hierarchical_b200 as hils
+    cfg = CONFIGS[name]
+    K = cfg["top_k"]
+    caches = []
+    for c in range(n_caches):
+        di = decode_inputs(seed=100 + c, device=dev, **cfg)
+        P, g, B, d = di.k_pages.shape
+        h = di.landmark_pages.shape[1]
+        kbar = torch.empty((P, h, d), dtype=torch.float32, device=dev)
+        hb = torch.empty((P, h), dtype=torch.float32, device=dev)
+        hils.summarize_paged(di.k_pages, di.landmark_pages, torch.arange(P, dtype=torch.int32, device=dev),
+                             kbar, hb)
+        call = hils.Decode(cfg["batch"], h, g, d, di.max_chunks, K, torch.bfloat16, device=dev)
+        out = torch.empty_like(di.q)
+        del di.landmark_pages
+        caches.append((di, kbar, hb, call, out))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(s):
+        for (di, kbar, hb, call, out) in caches:  # warm up outside capture
+            call(di.q, di.k_pages, di.v_pages, kbar, hb, di.block_table, di.seq_lens, out=out)
+    torch.cuda.synchronize()
+    for (di, kbar, hb, call, out) in caches:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            call(di.q, di.k_pages, di.v_pages, kbar, hb, di.block_table, di.seq_lens, out=out)
+        graphs.append(gr)
+    for gr in graphs:
+        gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for r in range(reps):
+        graphs[r % len(graphs)].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    for (di, kbar, hb, call, out) in caches:
+        assert call.device_status() == 0
+    alg, kv_only = decode_bytes(cfg)
+    del graphs, caches
+    torch.cuda.empty_cache()
+    return dict(ms=ms, tok_s=cfg["batch"] / (ms * 1e-3), gbs=alg / (ms * 1e-3) / 1e9, bytes=alg,
+                kv_bytes=kv_only)
+
+
+def run_ours(args):
+    ws_world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    hbm, bf16_peak, bf16_sus, peak_src = load_peaks()
+    pre = run_prefill(args, ws_world, rank, local)
+    dec = {}
+    if not args.no_decode:
+        for name, nc in (("decode_32k", 3), ("decode_128k", 1), ("decode_512k", 1)):
+            r = run_decode(name, nc, torch.device("cuda", local))
+            dec[name] = r
+    cpu = cpu_baseline(args.cpu_seconds) if (rank == 0 and ws_world == 1 and not args.no_cpu) else None
+    if ws_world > 1:
+        torch.distributed.barrier()
+    if rank != 0:
+        torch.distributed.destroy_process_group()
+        return
+    flops = pre["flops"]
+    value = ws_world * flops / (pre["ms_step"] * 1e-3) / 1e12
+    att_tflops = flops / (pre["ms_att"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": ws_world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(pre["ms_step"], 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill_345m: batch 4, 16 heads (MHA), N 8192, d 64, chunk 64, top-k 16, "
+                               "bf16 N(0,1) Q/K/V/landmarks, 8 needles per head",
+                   "global_batch": PREFILL["batch"] * ws_world, "seq_len": PREFILL["seq_len"],
+                   "parallelism": f"replicas x{ws_world}", "l2": "flushed (256 MB write) between steps",
+                   "algorithmic_gflop_per_step": round(flops / 1e9, 3)},
+        "stage_ms": {"summarize": round(pre["ms_summ"], 4), "select": round(pre["ms_sel"], 4),
+                     "attend_selected": round(pre["ms_att"], 4)},
+        "roofline": {"bound": "tensor", "kernel": "attend_selected (selected + own chunk attention, fusion)",
+                     "achieved": round(att_tflops, 3), "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": round(att_tflops / bf16_peak, 5), "peak_source": f"{peak_src} bf16 burst",
+                     "traffic": args.traffic},
+        "e2e": {"value": round(ws_world * flops / (pre["ms_e2e"] * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                "ms_per_step": round(pre["ms_e2e"], 3), "h2d_bytes_per_step": pre["h2d"],
+                "d2h_bytes_per_step": pre["d2h"]},
+        "gpu_launches": pre["launches_per_step"] * args.steps,
+        "clocks": pre["clocks"],
+    }
+    if dec:
+        line["decode"] = {
+            k: {"tok_s": round(r["tok_s"], 1), "us_per_step": round(r["ms"] * 1e3, 2),
+                "alg_bytes": int(r["bytes"]), "kv_bytes": int(r["kv_bytes"]),
+                "achieved_gbs": round(r["gbs"], 1), "frac_hbm": round(r["gbs"] / hbm, 4),
+                "timing": "CUDA-graph replay, 2 kernels per step"}
+            for k, r in dec.items()}
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    if ws_world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, bounded sample per step."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(per_step / 4)
+    vals = [cpu_baseline(per_step) for _ in range(args.steps)]
+    value = statistics.median(v["value"] for v in vals)
+    flops = algorithmic_flops(PREFILL["batch"], PREFILL["heads_q"], PREFILL["seq_len"], PREFILL["head_dim"],
+                              PREFILL["top_k"])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "prefill_345m: batch 4, 16 heads (MHA), N 8192, d 64, chunk 64, top-k 16",
+                   "global_batch": PREFILL["batch"], "seq_len": PREFILL["seq_len"], "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": vals[-1]["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the attention kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,259 @@
+"""ctypes binding of libhils.so (argument marshalling only).
+
+Every function takes torch tensors that already live on the GPU, checks their
+dtype, shape and contiguity, and passes raw pointers to the C ABI declared in
+include/hils.h.  All arithmetic happens in the CUDA kernels; there is no
+fallback: if the library is missing or the tensors are on the CPU, the call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhils.so")
+
+HILS_F32, HILS_BF16 = 0, 1
+OP_SELECT, OP_ATTEND, OP_DECODE, OP_ATTEND_SELECTED = 0, 1, 2, 3
+STATUS = {
+    0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED", 3: "HILS_ERR_WORKSPACE",
+    4: "HILS_ERR_CUDA", 5: "HILS_ERR_DEVICE_CHECK", 6: "HILS_ERR_DEVICE_TIMEOUT",
+}
+
+
+class HilsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("chunk", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib():
+    """Loads libhils.so once; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libhils.so not built ({LIB_PATH}); run "
+                           "`python -m chunk_wise_hierarchical_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    S = ctypes.POINTER(Shape)
+    i32, sz = ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "hils_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hils_abi_version": (i32, []),
+        "hils_workspace_size": (i32, [S, i32, ctypes.POINTER(sz)]),
+        "hils_summarize": (i32, [S, _P, _P, _P, _P, _P]),
+        "hils_summarize_paged": (i32, [S, _P, _P, _P, i32, i32, _P, _P, _P]),
+        "hils_select": (i32, [S, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "hils_attend": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "hils_attend_selected": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "hils_decode": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
+        "hils_device_status": (i32, [_P, _P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_decode",
+            "hils_device_status", "hils_select", "hils_status_string", "hils_summarize",
+            "hils_summarize_paged", "hils_workspace_size"]
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HILS_BF16
+    if t.dtype == torch.float32:
+        return HILS_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise HilsError(st, where)
+
+
+def make_shape(batch, heads_q, heads_kv, head_dim, seq_len, top_k, dtype, chunk=64, scale=0.0):
+    return Shape(batch, heads_q, heads_kv, head_dim, seq_len, chunk, top_k, float(scale or 0.0), dtype)
+
+
+def workspace_size(shape: Shape, op: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().hils_workspace_size(ctypes.byref(shape), op, ctypes.byref(out)), "hils_workspace_size")
+    return out.value
+
+
+def new_workspace(shape: Shape, op: int, device) -> torch.Tensor:
+    """Zero-filled workspace (the error word must start cleared)."""
+    n = workspace_size(shape, op)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def summarize(k, landmark, scale=None, stream=None):
+    """kbar [b,h,C,d] fp32, hbias [b,h,C] fp32 of every complete chunk."""
+    b, g, n, d = k.shape
+    h = landmark.shape[1]
+    c = n // 64
+    if landmark.shape != (b, h, c, d) or landmark.dtype != k.dtype:
+        raise ValueError("landmark must be [b, h, seq_len // 64, d] with k's dtype")
+    sh = make_shape(b, h, g, d, n, 0, _dt(k), scale=scale or 0.0)
+    kbar = torch.empty((b, h, c, d), dtype=torch.float32, device=k.device)
+    hb = torch.empty((b, h, c), dtype=torch.float32, device=k.device)
+    _check(lib().hils_summarize(ctypes.byref(sh), _ptr(k), _ptr(landmark), _ptr(kbar), _ptr(hb),
+                                _stream(stream)), "hils_summarize")
+    return kbar, hb
+
+
+def summarize_paged(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages, scale=None, stream=None):
+    """Writes the summaries of the listed pages into kbar_pages / hbias_pages."""
+    n_pages, g, chunk, d = k_pages.shape
+    h = landmark_pages.shape[1]
+    if page_ids.dtype != torch.int32:
+        raise TypeError("page_ids must be int32")
+    sh = make_shape(0, h, g, d, 0, 0, _dt(k_pages), chunk=chunk, scale=scale or 0.0)
+    _check(lib().hils_summarize_paged(ctypes.byref(sh), _ptr(k_pages), _ptr(landmark_pages), _ptr(page_ids),
+                                      int(page_ids.numel()), int(n_pages), _ptr(kbar_pages),
+                                      _ptr(hbias_pages), _stream(stream)), "hils_summarize_paged")
+
+
+def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True):
+    """topk_idx [b,g,N,K] int32 and (optionally) topk_score [b,h,N,K] fp32."""
+    b, h, n, d = q.shape
+    sh = make_shape(b, h, heads_kv, d, n, top_k, _dt(q), scale=scale or 0.0)
+    idx = torch.empty((b, heads_kv, n, top_k), dtype=torch.int32, device=q.device)
+    sc = torch.empty((b, h, n, top_k), dtype=torch.float32, device=q.device) if with_scores else None
+    ws = new_workspace(sh, OP_SELECT, q.device)
+    _check(lib().hils_select(ctypes.byref(sh), _ptr(q), _ptr(kbar), _ptr(hbias), _ptr(idx), _ptr(sc),
+                             _ptr(ws), ws.numel(), _stream(stream)), "hils_select")
+    return idx, sc
+
+
+class Prefill:
+    """Reusable prefill call: holds the workspace for one shape."""
+
+    def __init__(self, batch, heads_q, heads_kv, seq_len, head_dim, top_k, dtype, scale=None, device="cuda"):
+        self.shape = make_shape(batch, heads_q, heads_kv, head_dim, seq_len, top_k,
+                                HILS_BF16 if dtype in (torch.bfloat16, "bf16") else HILS_F32,
+                                scale=scale or 0.0)
+        self.ws = new_workspace(self.shape, OP_ATTEND, device)
+
+    def __call__(self, q, k, v, landmark, out=None, topk_idx=None, stream=None):
+        s = self.shape
+        if q.shape != (s.batch, s.heads_q, s.seq_len, s.head_dim) or _dt(q) != s.dtype:
+            raise ValueError("q does not match the prepared shape")
+        for t in (k, v, landmark):
+            if t.dtype != q.dtype:
+                raise TypeError("q, k, v and landmark must share a dtype")
+        if out is None:
+            out = torch.empty_like(q)
+        _check(lib().hils_attend(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(landmark), _ptr(out),
+                                 _ptr(topk_idx), _ptr(self.ws), self.ws.numel(), _stream(stream)),
+               "hils_attend")
+        return out
+
+    def device_status(self, stream=None):
+        return lib().hils_device_status(_ptr(self.ws), _stream(stream))
+
+
+def attend(q, k, v, landmark, top_k, scale=None, stream=None, return_idx=False):
+    """HiLS prefill forward; returns out (and topk_idx if asked)."""
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    call = Prefill(b, h, g, n, d, top_k, q.dtype, scale=scale, device=q.device)
+    idx = torch.empty((b, g, n, top_k), dtype=torch.int32, device=q.device) if return_idx else None
+    out = call(q, k, v, landmark, topk_idx=idx, stream=stream)
+    return (out, idx) if return_idx else out
+
+
+def attend_selected(q, k, v, topk_idx, topk_score, scale=None, out=None, ws=None, stream=None):
+    """Attention + fusion for a given selection (topk_idx [b,g,N,K], topk_score [b,h,N,K])."""
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    K = topk_idx.shape[-1]
+    sh = make_shape(b, h, g, d, n, K, _dt(q), scale=scale or 0.0)
+    if topk_idx.dtype != torch.int32 or topk_score.dtype != torch.float32:
+        raise TypeError("topk_idx must be int32 and topk_score fp32")
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = new_workspace(sh, OP_ATTEND_SELECTED, q.device)
+    _check(lib().hils_attend_selected(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx),
+                                      _ptr(topk_score), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "hils_attend_selected")
+    return out
+
+
+class Decode:
+    """Reusable decode call for a paged cache of `max_chunks` chunks per sequence."""
+
+    def __init__(self, batch, heads_q, heads_kv, head_dim, max_chunks, top_k, dtype, scale=None,
+                 device="cuda"):
+        self.max_chunks = max_chunks
+        self.shape = make_shape(batch, heads_q, heads_kv, head_dim, max_chunks * 64, top_k,
+                                HILS_BF16 if dtype in (torch.bfloat16, "bf16") else HILS_F32,
+                                scale=scale or 0.0)
+        self.ws = new_workspace(self.shape, OP_DECODE, device)
+
+    def __call__(self, q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, out=None,
+                 topk_idx=None, stream=None):
+        s = self.shape
+        if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+            raise TypeError("block_table and seq_lens must be int32")
+        if block_table.shape != (s.batch, self.max_chunks):
+            raise ValueError("block_table must be [batch, max_chunks]")
+        if out is None:
+            out = torch.empty_like(q)
+        _check(lib().hils_decode(ctypes.byref(s), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kbar_pages),
+                                 _ptr(hbias_pages), _ptr(block_table), self.max_chunks, _ptr(seq_lens),
+                                 int(k_pages.shape[0]), _ptr(out), _ptr(topk_idx), _ptr(self.ws),
+                                 self.ws.numel(), _stream(stream)), "hils_decode")
+        return out
+
+    def device_status(self, stream=None):
+        return lib().hils_device_status(_ptr(self.ws), _stream(stream))
+
+
+def decode(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, top_k, scale=None,
+           stream=None, return_idx=False):
+    b, h, d = q.shape
+    g = k_pages.shape[1]
+    call = Decode(b, h, g, d, block_table.shape[1], top_k, q.dtype, scale=scale, device=q.device)
+    idx = torch.empty((b, g, top_k), dtype=torch.int32, device=q.device) if return_idx else None
+    out = call(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, topk_idx=idx,
+               stream=stream)
+    return (out, idx) if return_idx else out

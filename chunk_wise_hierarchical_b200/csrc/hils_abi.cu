@@ -1,0 +1,276 @@
+// C ABI of libhils.so: argument validation, workspace layout and dispatch.
+// Every entry point checks its arguments on the host, then enqueues kernels on
+// the caller's stream; nothing here allocates device memory or synchronises
+// (except hils_device_status).
+#include <cmath>
+#include <cstring>
+
+#include "../../include/hils.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeader = 256;  // error word + reserved
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hils_status check_shape(const hils_shape* s, bool need_seq) {
+  if (!s) return HILS_ERR_INVALID_ARG;
+  if (s->batch < 0 || s->heads_q <= 0 || s->heads_kv <= 0 || s->head_dim <= 0 || s->seq_len < 0 ||
+      s->chunk <= 0 || s->top_k < 0)
+    return HILS_ERR_INVALID_ARG;
+  if (s->heads_q % s->heads_kv != 0) return HILS_ERR_INVALID_ARG;
+  if (!std::isfinite(s->scale)) return HILS_ERR_INVALID_ARG;
+  if (s->dtype != HILS_F32 && s->dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+  const int grp = s->heads_q / s->heads_kv;
+  if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return HILS_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return HILS_ERR_UNSUPPORTED;
+  if (s->chunk != hils::kChunk) return HILS_ERR_UNSUPPORTED;
+  if (s->top_k > hils::kMaxTopK) return HILS_ERR_UNSUPPORTED;
+  (void)need_seq;
+  return HILS_OK;
+}
+
+float eff_scale(const hils_shape* s) {
+  return s->scale == 0.f ? 1.0f / std::sqrt((float)s->head_dim) : s->scale;
+}
+
+struct AttendLayout {
+  size_t kbar, hbias, idx, ssel, total;
+};
+AttendLayout attend_layout(const hils_shape* s) {
+  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, n = s->seq_len, d = s->head_dim;
+  const size_t C = n / s->chunk, K = s->top_k;
+  AttendLayout L;
+  size_t off = kHeader;
+  L.kbar = off; off = align_up(off + b * h * C * d * 4);
+  L.hbias = off; off = align_up(off + b * h * C * 4);
+  L.idx = off; off = align_up(off + b * g * n * K * 4);
+  L.ssel = off; off = align_up(off + b * h * n * K * 4);
+  L.total = off;
+  return L;
+}
+
+struct DecodeLayout {
+  size_t keys, idx, ssel, total;
+};
+DecodeLayout decode_layout(const hils_shape* s) {
+  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k;
+  const size_t cmax = (s->seq_len + s->chunk - 1) / s->chunk;
+  DecodeLayout L;
+  size_t off = kHeader;
+  L.keys = off; off = align_up(off + b * g * cmax * 8);
+  L.idx = off; off = align_up(off + b * g * K * 4);
+  L.ssel = off; off = align_up(off + b * h * K * 4);
+  L.total = off;
+  return L;
+}
+
+hils_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* hils_status_string(int status) {
+  switch (status) {
+    case HILS_OK: return "ok";
+    case HILS_ERR_INVALID_ARG: return "invalid argument";
+    case HILS_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case HILS_ERR_WORKSPACE: return "workspace missing or too small";
+    case HILS_ERR_CUDA: return "CUDA error";
+    case HILS_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case HILS_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t hils_abi_version(void) { return 1; }
+
+hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) {
+  if (!bytes) return HILS_ERR_INVALID_ARG;
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  switch (op) {
+    case HILS_OP_SELECT: *bytes = 0; return HILS_OK;
+    case HILS_OP_ATTEND: *bytes = attend_layout(s).total; return HILS_OK;
+    case HILS_OP_DECODE: *bytes = decode_layout(s).total; return HILS_OK;
+    case HILS_OP_ATTEND_SELECTED: *bytes = kHeader; return HILS_OK;
+  }
+  return HILS_ERR_INVALID_ARG;
+}
+
+hils_status hils_summarize(const hils_shape* s, const void* k, const void* landmark_q, float* kbar,
+                           float* hbias, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  const int C = s->seq_len / s->chunk;
+  if ((size_t)s->batch * C == 0) return HILS_OK;
+  if (!k || !landmark_q || !kbar || !hbias) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(landmark_q) || !aligned16(kbar)) return HILS_ERR_INVALID_ARG;
+  hils::SummarizeArgs a{};
+  a.k = k; a.lm = landmark_q; a.kbar = kbar; a.hbias = hbias;
+  a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
+  a.n_chunks = C; a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
+  a.page_ids = nullptr;
+  return cuda_status(hils::run_summarize(a, (cudaStream_t)stream));
+}
+
+hils_status hils_summarize_paged(const hils_shape* s, const void* k_pages, const void* landmark_pages,
+                                 const int32_t* page_ids, int32_t n_listed, int32_t n_pages,
+                                 float* kbar_pages, float* hbias_pages, void* stream) {
+  hils_status st = check_shape(s, false);
+  if (st != HILS_OK) return st;
+  if (n_listed < 0 || n_pages < 0) return HILS_ERR_INVALID_ARG;
+  if (n_listed == 0) return HILS_OK;
+  if (!k_pages || !landmark_pages || !page_ids || !kbar_pages || !hbias_pages) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(k_pages) || !aligned16(landmark_pages) || !aligned16(kbar_pages)) return HILS_ERR_INVALID_ARG;
+  hils::SummarizeArgs a{};
+  a.k = k_pages; a.lm = landmark_pages; a.kbar = kbar_pages; a.hbias = hbias_pages;
+  a.b = 0; a.h = s->heads_q; a.g = s->heads_kv; a.n = 0; a.d = s->head_dim; a.n_chunks = 0;
+  a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
+  a.page_ids = page_ids; a.n_listed = n_listed; a.n_pages = n_pages;
+  return cuda_status(hils::run_summarize(a, (cudaStream_t)stream));
+}
+
+hils_status hils_select(const hils_shape* s, const void* q, const float* kbar, const float* hbias,
+                        int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if ((size_t)s->batch * s->seq_len * s->top_k == 0) return HILS_OK;
+  const int C = s->seq_len / s->chunk;
+  if (!q || !topk_idx || (C > 0 && (!kbar || !hbias))) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q)) return HILS_ERR_INVALID_ARG;
+  hils::SelectArgs a{};
+  a.q = q; a.kbar = kbar; a.hbias = hbias; a.idx = topk_idx; a.score = topk_score;
+  a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
+  a.n_chunks = C; a.top_k = s->top_k; a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
+  return cuda_status(hils::run_select_simt(a, (cudaStream_t)stream));
+}
+
+hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const void* v,
+                        const void* landmark_q, void* out, int32_t* topk_idx_out, void* ws,
+                        size_t ws_bytes, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if ((size_t)s->batch * s->seq_len == 0) return HILS_OK;
+  const int C = s->seq_len / s->chunk;
+  if (!q || !k || !v || !out || (C > 0 && !landmark_q)) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (C > 0 && !aligned16(landmark_q)))
+    return HILS_ERR_INVALID_ARG;
+  const AttendLayout L = attend_layout(s);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* w = static_cast<char*>(ws);
+  float* kbar = reinterpret_cast<float*>(w + L.kbar);
+  float* hbias = reinterpret_cast<float*>(w + L.hbias);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  float* ssel = reinterpret_cast<float*>(w + L.ssel);
+  const bool bf16 = s->dtype == HILS_BF16;
+  const float scale = eff_scale(s);
+
+  if (C > 0) {
+    hils::SummarizeArgs sa{};
+    sa.k = k; sa.lm = landmark_q; sa.kbar = kbar; sa.hbias = hbias;
+    sa.b = s->batch; sa.h = s->heads_q; sa.g = s->heads_kv; sa.n = s->seq_len; sa.d = s->head_dim;
+    sa.n_chunks = C; sa.scale = scale; sa.bf16 = bf16; sa.page_ids = nullptr;
+    if (hils::run_summarize(sa, cs) != cudaSuccess) return HILS_ERR_CUDA;
+  }
+  if (s->top_k > 0) {
+    hils::SelectArgs se{};
+    se.q = q; se.kbar = kbar; se.hbias = hbias; se.idx = idx; se.score = ssel;
+    se.b = s->batch; se.h = s->heads_q; se.g = s->heads_kv; se.n = s->seq_len; se.d = s->head_dim;
+    se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16;
+    if (hils::run_select_simt(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
+  }
+  hils::AttendRowsArgs ar{};
+  ar.q = q; ar.k = k; ar.v = v; ar.idx = idx; ar.ssel = ssel; ar.out = out;
+  ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = reinterpret_cast<unsigned*>(w);
+  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
+  ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = scale; ar.bf16 = bf16;
+  ar.paged = false;
+  return cuda_status(hils::run_attend_rows(ar, cs));
+}
+
+hils_status hils_attend_selected(const hils_shape* s, const void* q, const void* k, const void* v,
+                                 const int32_t* topk_idx, const float* topk_score, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if ((size_t)s->batch * s->seq_len == 0) return HILS_OK;
+  if (!q || !k || !v || !out || (s->top_k > 0 && (!topk_idx || !topk_score))) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HILS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  hils::AttendRowsArgs ar{};
+  ar.q = q; ar.k = k; ar.v = v; ar.idx = topk_idx; ar.ssel = topk_score; ar.out = out;
+  ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = reinterpret_cast<unsigned*>(ws);
+  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
+  ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = eff_scale(s);
+  ar.bf16 = s->dtype == HILS_BF16; ar.paged = false;
+  return cuda_status(hils::run_attend_rows(ar, (cudaStream_t)stream));
+}
+
+hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages, const void* v_pages,
+                        const float* kbar_pages, const float* hbias_pages, const int32_t* block_table,
+                        int32_t max_chunks, const int32_t* seq_lens, int32_t n_pages, void* out,
+                        int32_t* topk_idx_out, void* ws, size_t ws_bytes, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if (s->batch == 0) return HILS_OK;
+  if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
+  if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
+  if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
+    return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(kbar_pages) ||
+      !aligned16(out))
+    return HILS_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(s);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  cudaStream_t cs = (cudaStream_t)stream;
+  char* w = static_cast<char*>(ws);
+  unsigned* err = reinterpret_cast<unsigned*>(w);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  float* ssel = reinterpret_cast<float*>(w + L.ssel);
+  const bool bf16 = s->dtype == HILS_BF16;
+  const float scale = eff_scale(s);
+
+  hils::DecodeSelectArgs ds{};
+  ds.q = q; ds.kbar_pages = kbar_pages; ds.hbias_pages = hbias_pages; ds.block_table = block_table;
+  ds.seq_lens = seq_lens; ds.keys = reinterpret_cast<unsigned long long*>(w + L.keys);
+  ds.idx = idx; ds.score = ssel; ds.err = err;
+  ds.b = s->batch; ds.h = s->heads_q; ds.g = s->heads_kv; ds.d = s->head_dim;
+  ds.max_chunks = max_chunks; ds.top_k = s->top_k; ds.n_pages = n_pages; ds.scale = scale; ds.bf16 = bf16;
+  if (s->top_k > 0 && hils::run_decode_select(ds, cs) != cudaSuccess) return HILS_ERR_CUDA;
+
+  hils::AttendRowsArgs ar{};
+  ar.q = q; ar.k = k_pages; ar.v = v_pages; ar.idx = idx; ar.ssel = ssel; ar.out = out;
+  ar.block_table = block_table; ar.seq_lens = seq_lens; ar.err = err;
+  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = 1; ar.d = s->head_dim;
+  ar.top_k = s->top_k; ar.max_chunks = max_chunks; ar.n_pages = n_pages; ar.scale = scale;
+  ar.bf16 = bf16; ar.paged = true;
+  return cuda_status(hils::run_attend_rows(ar, cs));
+}
+
+hils_status hils_device_status(void* ws, void* stream) {
+  if (!ws) return HILS_ERR_INVALID_ARG;
+  cudaStream_t cs = (cudaStream_t)stream;
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return HILS_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return HILS_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(word), cs) != cudaSuccess) return HILS_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return HILS_ERR_CUDA;
+  }
+  if (word & hils::kErrTimeout) return HILS_ERR_DEVICE_TIMEOUT;
+  if (word & hils::kErrBadPage) return HILS_ERR_DEVICE_CHECK;
+  return HILS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Host-side launch interface of the HiLS kernels (one struct per kernel family).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hils {
+
+struct SummarizeArgs {
+  const void* k;          // [b,g,N,d] or pages [P,g,B,d]
+  const void* lm;         // [b,h,C,d] or pages [P,h,d]
+  float* kbar;            // [b,h,C,d] or [P,h,d]
+  float* hbias;           // [b,h,C]   or [P,h]
+  int b, h, g, n, d, n_chunks;
+  float scale;
+  bool bf16;
+  const int32_t* page_ids;  // nullptr: contiguous mode
+  int n_listed, n_pages;
+};
+cudaError_t run_summarize(const SummarizeArgs& a, cudaStream_t st);
+
+struct SelectArgs {
+  const void* q;          // [b,h,N,d]
+  const float* kbar;      // [b,h,C,d]
+  const float* hbias;     // [b,h,C]
+  int32_t* idx;           // [b,g,N,K]
+  float* score;           // [b,h,N,K] or nullptr
+  int b, h, g, n, d, n_chunks, top_k;
+  float scale;
+  bool bf16;
+};
+cudaError_t run_select_simt(const SelectArgs& a, cudaStream_t st);
+
+struct DecodeSelectArgs {
+  const void* q;               // [b,h,d]
+  const float* kbar_pages;     // [P,h,d]
+  const float* hbias_pages;    // [P,h]
+  const int32_t* block_table;  // [b,max_chunks]
+  const int32_t* seq_lens;     // [b]
+  unsigned long long* keys;    // workspace [b,g,max_chunks]
+  int32_t* idx;                // [b,g,K]
+  float* score;                // [b,h,K]
+  unsigned* err;
+  int b, h, g, d, max_chunks, top_k, n_pages;
+  float scale;
+  bool bf16;
+};
+cudaError_t run_decode_select(const DecodeSelectArgs& a, cudaStream_t st);
+
+// Row-wise attention + fusion (one warp per query and KV group).
+struct AttendRowsArgs {
+  const void* q;               // prefill [b,h,N,d]; decode [b,h,d]
+  const void* k;               // prefill [b,g,N,d]; decode pages [P,g,B,d]
+  const void* v;
+  const int32_t* idx;          // prefill [b,g,N,K]; decode [b,g,K]
+  const float* ssel;           // prefill [b,h,N,K]; decode [b,h,K]
+  void* out;                   // like q
+  const int32_t* block_table;  // decode only
+  const int32_t* seq_lens;     // decode only
+  unsigned* err;
+  int b, h, g, n, d, top_k, max_chunks, n_pages;
+  float scale;
+  bool bf16;
+  bool paged;                  // decode mode
+};
+cudaError_t run_attend_rows(const AttendRowsArgs& a, cudaStream_t st);
+
+}  // namespace hils

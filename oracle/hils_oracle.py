@@ -293,7 +293,8 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
     block_table[b, c] of the pools k_pages/v_pages [P,g,B,d].  The own chunk is
     floor((seq_len-1)/B); candidates are the complete chunks before it, scored
     with summaries computed here from landmark_pages [P,h,d].
-    Returns out [b,h,d] (zeros for seq_len <= 0) and idx [b,g,K].
+    Returns out [b,h,d] (zeros for seq_len <= 0), idx [b,g,K] and, per
+    sequence, the selection key [g, own] of its candidate chunks.
     """
     q64, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
     bt = np.asarray(block_table).astype(np.int64)
@@ -306,6 +307,7 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
     out = np.zeros((b, h, d))
     idx = np.full((b, g, top_k), -1, dtype=np.int64)
     shat_sel = np.full((b, h, top_k), -np.inf)
+    keys = {}
     for bi in range(b) if batches is None else batches:
         L = int(sl[bi])
         if L <= 0:
@@ -317,8 +319,9 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
         for c in range(own):
             kb, hb = summ[int(pages[c])]
             shat[:, c] = np.einsum("hd,hd->h", kb, q64[bi]) * sc + hb
-        sel, _ = select_topk(shat[None, :, None, :], g, top_k)
+        sel, key = select_topk(shat[None, :, None, :], g, top_k)
         idx[bi] = sel[0, :, 0]
+        keys[bi] = key[0, :, 0]
         own_page = int(bt[bi, own])
         n_own = L - own * chunk
         for hi in range(h):
@@ -337,4 +340,4 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
             w = np.array([math.exp(x - mx) for x, _ in terms])
             w /= w.sum()
             out[bi, hi] = sum(wi * o for wi, (_, o) in zip(w, terms))
-    return dict(out=out, idx=idx, shat_sel=shat_sel)
+    return dict(out=out, idx=idx, shat_sel=shat_sel, key=keys)

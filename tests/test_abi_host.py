@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_wise_hierarchical_b200 as hils
+from chunk_wise_hierarchical_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "hils.h")).read()
+    return sorted(set(re.findall(r"HILS_API[^;(]*?\b(hils_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = hils.lib()
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(hils.EXPORTED) == names
+
+
+def test_status_strings_and_version():
+    lib = hils.lib()
+    assert lib.hils_abi_version() == 1
+    for code in range(7):
+        assert lib.hils_status_string(code)
+    assert lib.hils_status_string(99) == b"unknown status"
+
+
+def _shape(**kw):
+    base = dict(batch=2, heads_q=8, heads_kv=2, head_dim=64, seq_len=1000, top_k=16, dtype=1)
+    base.update(kw)
+    return _abi.make_shape(base["batch"], base["heads_q"], base["heads_kv"], base["head_dim"],
+                           base["seq_len"], base["top_k"], base["dtype"],
+                           chunk=base.get("chunk", 64), scale=base.get("scale", 0.0))
+
+
+def test_workspace_sizes():
+    s = _shape()
+    n = _abi.workspace_size(s, _abi.OP_ATTEND)
+    C = 1000 // 64
+    need = 2 * 8 * C * 64 * 4 + 2 * 8 * C * 4 + 2 * 2 * 1000 * 16 * 4 + 2 * 8 * 1000 * 16 * 4
+    assert need <= n <= need + 6 * 256
+    assert _abi.workspace_size(s, _abi.OP_SELECT) == 0
+    assert _abi.workspace_size(s, _abi.OP_DECODE) >= 2 * 2 * 16 * 8
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), 2), (dict(chunk=32), 2), (dict(top_k=65), 2), (dict(heads_q=6, heads_kv=2), 2),
+    (dict(heads_q=7, heads_kv=2), 1), (dict(batch=-1), 1), (dict(dtype=5), 1), (dict(top_k=-1), 1),
+    (dict(scale=float("nan")), 1), (dict(heads_q=32, heads_kv=2), 2),
+])
+def test_shape_validation(kw, code):
+    s = _shape(**kw)
+    out = ctypes.c_size_t(0)
+    assert hils.lib().hils_workspace_size(ctypes.byref(s), 1, ctypes.byref(out)) == code
+
+
+def test_entry_points_reject_before_launch():
+    lib = hils.lib()
+    s = _shape()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below fails validation first
+    assert lib.hils_workspace_size(None, 1, ctypes.byref(ctypes.c_size_t())) == 1
+    assert lib.hils_attend(ctypes.byref(s), None, fake, fake, fake, fake, None, fake, 1 << 30, None) == 1
+    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, None, 0, None) == 3
+    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, fake, 16, None) == 3
+    assert lib.hils_attend(ctypes.byref(s), P((1 << 20) + 4), fake, fake, fake, fake, None, fake,
+                           1 << 30, None) == 1  # misaligned
+    assert lib.hils_select(ctypes.byref(s), fake, None, fake, fake, None, None, 0, None) == 1
+    assert lib.hils_summarize(ctypes.byref(s), fake, None, fake, fake, None) == 1
+    assert lib.hils_summarize_paged(ctypes.byref(s), fake, fake, fake, -1, 4, fake, fake, None) == 1
+    assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 0, fake, 4, fake, None,
+                           fake, 1 << 30, None) == 1
+    assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 100, fake, 4, fake, None,
+                           fake, 1 << 30, None) == 1  # more chunks than seq_len allows
+    assert lib.hils_device_status(None, None) == 1
+
+
+def test_empty_problems_are_no_ops():
+    lib = hils.lib()
+    P = ctypes.c_void_p
+    s0 = _shape(batch=0)
+    assert lib.hils_attend(ctypes.byref(s0), None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.hils_decode(ctypes.byref(s0), None, None, None, None, None, None, 0, None, 0, None, None,
+                           None, 0, None) == 0
+    s1 = _shape(seq_len=0)
+    assert lib.hils_attend(ctypes.byref(s1), None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.hils_summarize(ctypes.byref(s1), None, None, None, None, None) == 0
+    s2 = _shape(top_k=0)
+    assert lib.hils_select(ctypes.byref(s2), None, None, None, None, None, None, 0, None) == 0
+    assert lib.hils_summarize_paged(ctypes.byref(s2), P(16), P(16), P(16), 0, 4, P(16), P(16), None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 64, 64)
+    with pytest.raises((ValueError, RuntimeError)):
+        hils.attend(q, q, q, torch.zeros(1, 1, 1, 64), top_k=1)
