@@ -19,6 +19,9 @@ def check_indices(gpu_idx, key, top_k, gap=TIE_GAP):
     if top_k == 0:
         assert np.asarray(gpu_idx).size == 0
         return 0
+    if np.asarray(key).shape[-1] == 0:  # no complete chunk before any query
+        assert np.all(np.asarray(gpu_idx) == -1)
+        return 0
     gpu_idx = np.asarray(gpu_idx).reshape(-1, gpu_idx.shape[-1])
     key = np.asarray(key).reshape(-1, key.shape[-1])
     ties = 0
