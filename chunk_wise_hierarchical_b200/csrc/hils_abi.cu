@@ -72,6 +72,32 @@ DecodeLayout decode_layout(const hils_shape* s) {
 
 hils_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
 
+// Prefill attention + fusion for a selection: the tcgen05 kernel for bf16
+// inputs when its shared-memory plan fits the shape, else the row kernel.
+cudaError_t run_prefill_attention(const hils_shape* s, const void* q, const void* k, const void* v,
+                                  const int32_t* idx, const float* ssel, void* out, unsigned* err,
+                                  cudaStream_t cs) {
+  const bool bf16 = s->dtype == HILS_BF16;
+  const int G = s->heads_q / s->heads_kv;
+  if (bf16 && hils::attend_tc_supported(s->head_dim, G, s->top_k, s->seq_len)) {
+    hils::TcAttendArgs ta{};
+    ta.q = static_cast<const __nv_bfloat16*>(q);
+    ta.k = static_cast<const __nv_bfloat16*>(k);
+    ta.v = static_cast<const __nv_bfloat16*>(v);
+    ta.idx = idx; ta.ssel = ssel; ta.out = static_cast<__nv_bfloat16*>(out); ta.err = err;
+    ta.b = s->batch; ta.h = s->heads_q; ta.g = s->heads_kv; ta.n = s->seq_len; ta.top_k = s->top_k;
+    ta.scale = eff_scale(s);
+    return hils::run_attend_tc(ta, s->head_dim, cs);
+  }
+  hils::AttendRowsArgs ar{};
+  ar.q = q; ar.k = k; ar.v = v; ar.idx = idx; ar.ssel = ssel; ar.out = out;
+  ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = err;
+  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
+  ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = eff_scale(s); ar.bf16 = bf16;
+  ar.paged = false;
+  return hils::run_attend_rows(ar, cs);
+}
+
 }  // namespace
 
 extern "C" {
@@ -189,13 +215,7 @@ hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const
     se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16;
     if (hils::run_select_simt(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
   }
-  hils::AttendRowsArgs ar{};
-  ar.q = q; ar.k = k; ar.v = v; ar.idx = idx; ar.ssel = ssel; ar.out = out;
-  ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = reinterpret_cast<unsigned*>(w);
-  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
-  ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = scale; ar.bf16 = bf16;
-  ar.paged = false;
-  return cuda_status(hils::run_attend_rows(ar, cs));
+  return cuda_status(run_prefill_attention(s, q, k, v, idx, ssel, out, reinterpret_cast<unsigned*>(w), cs));
 }
 
 hils_status hils_attend_selected(const hils_shape* s, const void* q, const void* k, const void* v,
@@ -207,13 +227,8 @@ hils_status hils_attend_selected(const hils_shape* s, const void* q, const void*
   if (!q || !k || !v || !out || (s->top_k > 0 && (!topk_idx || !topk_score))) return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HILS_ERR_INVALID_ARG;
   if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
-  hils::AttendRowsArgs ar{};
-  ar.q = q; ar.k = k; ar.v = v; ar.idx = topk_idx; ar.ssel = topk_score; ar.out = out;
-  ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = reinterpret_cast<unsigned*>(ws);
-  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
-  ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = eff_scale(s);
-  ar.bf16 = s->dtype == HILS_BF16; ar.paged = false;
-  return cuda_status(hils::run_attend_rows(ar, (cudaStream_t)stream));
+  return cuda_status(run_prefill_attention(s, q, k, v, topk_idx, topk_score, out,
+                                           reinterpret_cast<unsigned*>(ws), (cudaStream_t)stream));
 }
 
 hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages, const void* v_pages,

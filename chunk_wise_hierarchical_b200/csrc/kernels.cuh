@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <cuda_bf16.h>
 
 namespace hils {
 
@@ -65,5 +66,22 @@ struct AttendRowsArgs {
   bool paged;                  // decode mode
 };
 cudaError_t run_attend_rows(const AttendRowsArgs& a, cudaStream_t st);
+
+// Tensor-core prefill attention + fusion for a given selection (bf16 only).
+struct TcAttendArgs {
+  const __nv_bfloat16* q;      // [b,h,N,d]
+  const __nv_bfloat16* k;      // [b,g,N,d]
+  const __nv_bfloat16* v;
+  const int32_t* idx;          // [b,g,N,K]
+  const float* ssel;           // [b,h,N,K]
+  __nv_bfloat16* out;          // [b,h,N,d]
+  unsigned* err;
+  int b, h, g, n, top_k;
+  float scale;
+  int qb;                      // queries per CTA (set by the launcher)
+  int n_cand_max;              // N / chunk (set by the launcher)
+};
+bool attend_tc_supported(int d, int G, int K, int N);
+cudaError_t run_attend_tc(const TcAttendArgs& a, int d, cudaStream_t st);
 
 }  // namespace hils
