@@ -319,12 +319,18 @@ def run_ours(args):
     ws_world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
     hbm, bf16_peak, bf16_sus, peak_src = load_peaks()
-    pre = run_prefill(args, ws_world, rank, local)
     dec = {}
     if not args.no_decode:
-        for name, nc in (("decode_32k", 3), ("decode_128k", 1), ("decode_512k", 1)):
-            r = run_decode(name, nc, torch.device("cuda", local))
-            dec[name] = r
+        for name in args.decode_configs.split(","):
+            nc = 3 if name == "decode_32k" else 1   # 3 rotating caches keep 32K out of L2
+            dec[name] = run_decode(name, nc, torch.device("cuda", local))
+    if args.decode_only:
+        if rank == 0:
+            print(json.dumps({"decode": {k: {"us_per_step": round(r["ms"] * 1e3, 2),
+                                             "tok_s": round(r["tok_s"], 1),
+                                             "frac_hbm": round(r["gbs"] / hbm, 4)} for k, r in dec.items()}}))
+        return
+    pre = run_prefill(args, ws_world, rank, local)
     cpu = cpu_baseline(args.cpu_seconds) if (rank == 0 and ws_world == 1 and not args.no_cpu) else None
     if ws_world > 1:
         torch.distributed.barrier()
@@ -412,6 +418,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="time only the decode configurations")
+    ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,

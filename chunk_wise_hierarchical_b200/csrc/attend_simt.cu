@@ -1,7 +1,7 @@
 // Row-wise HiLS attention on CUDA cores: intra-chunk softmax attention over
 // each selected chunk and the own causal chunk, then the inter-chunk fusion
-// (HiLS notes, section 5.3; Tide digest, Figure 3).  Used for fp32 inputs,
-// for decode, and as the reference-shaped path for any shape.
+// (HiLS notes, section 5.3; Tide digest, Figure 3).  Used for fp32 prefill
+// and for shapes outside the tensor-core kernel's shared-memory plan.
 //
 // One warp per (sequence, KV group, query): lane j owns keys j and j+32 of a
 // chunk, and d/32 output columns.  The group's G query heads share every key
@@ -10,10 +10,6 @@
 // weights chunk c by exp(shat_c - M) / Z' and the own chunk by
 // exp(LSE_own - M) / Z', with M the max of all log-masses and Z' their
 // shifted sum.
-//
-// Also here: the decode selection kernel (one CTA per sequence and KV group)
-// that scores every earlier chunk against the paged summary cache and keeps
-// the Top-K by repeated block-wide arg-max.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -216,111 +212,6 @@ static cudaError_t rows_by_group(const AttendRowsArgs& a, cudaStream_t st) {
 cudaError_t run_attend_rows(const AttendRowsArgs& a, cudaStream_t st) {
   if (a.bf16) return a.d == 64 ? rows_by_group<__nv_bfloat16, 64>(a, st) : rows_by_group<__nv_bfloat16, 128>(a, st);
   return a.d == 64 ? rows_by_group<float, 64>(a, st) : rows_by_group<float, 128>(a, st);
-}
-
-// ---------------------------------------------------------------------------
-// Decode selection: one CTA per (sequence, KV group).
-// ---------------------------------------------------------------------------
-constexpr int kDecSelThreads = 256;
-
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(DecodeSelectArgs a) {
-  __shared__ __align__(16) float qS[G * D];
-  __shared__ unsigned long long wbest[kDecSelThreads / 32];
-  __shared__ int sel[kMaxTopK];
-  const int t = threadIdx.x;
-  const int gi = blockIdx.x % a.g;
-  const int bi = blockIdx.x / a.g;
-  const int K = a.top_k;
-  const int L = a.seq_lens[bi];
-  const int own = L > 0 ? (L - 1) / kChunk : 0;
-  const int n_cand = min(own, a.max_chunks);
-  for (int x = t; x < G * D; x += blockDim.x) {
-    const int hh = x / D, e = x % D;
-    qS[x] = to_f(static_cast<const T*>(a.q)[((size_t)bi * a.h + gi * G + hh) * D + e]);
-  }
-  __syncthreads();
-  unsigned long long* keys = a.keys + ((size_t)bi * a.g + gi) * a.max_chunks;
-  const int32_t* bt = a.block_table + (size_t)bi * a.max_chunks;
-  for (int c = t; c < n_cand; c += blockDim.x) {
-    const int p = bt[c];
-    unsigned long long key = 0;
-    if (p < 0 || p >= a.n_pages) {
-      set_error(a.err, kErrBadPage);
-    } else {
-      float best = -INFINITY;
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float* kb = a.kbar_pages + ((size_t)p * a.h + gi * G + hh) * D;
-        float acc = 0.f;
-#pragma unroll 4
-        for (int e = 0; e < D; e += 4) {
-          const float4 kv = *reinterpret_cast<const float4*>(kb + e);
-          const float4 qv = *reinterpret_cast<const float4*>(qS + hh * D + e);
-          acc = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, acc))));
-        }
-        best = fmaxf(best, fmaf(acc, a.scale, a.hbias_pages[(size_t)p * a.h + gi * G + hh]));
-      }
-      key = pack_key(best, c);
-    }
-    keys[c] = key;
-  }
-  // K rounds of block arg-max; the owner thread of the winning chunk clears it
-  for (int s = 0; s < K; ++s) {
-    unsigned long long best = 0;
-    for (int c = t; c < n_cand; c += blockDim.x) best = keys[c] > best ? keys[c] : best;
-    best = warp_max_u64(best);
-    if ((t & 31) == 0) wbest[t >> 5] = best;
-    __syncthreads();
-    if (t < 32) {
-      unsigned long long v = t < kDecSelThreads / 32 ? wbest[t] : 0;
-      v = warp_max_u64(v);
-      if (t == 0) sel[s] = v ? key_chunk(v) : -1;
-    }
-    __syncthreads();
-    const int c = sel[s];
-    if (c >= 0 && (c % blockDim.x) == t) keys[c] = 0;
-    __syncthreads();
-  }
-  // outputs: indices and each head's own score of the selected chunks
-  for (int x = t; x < K * G; x += blockDim.x) {
-    const int s = x / G, hh = x % G;
-    const int c = sel[s];
-    float sc = -INFINITY;
-    if (c >= 0) {
-      const int p = bt[c];
-      const float* kb = a.kbar_pages + ((size_t)p * a.h + gi * G + hh) * D;
-      float acc = 0.f;
-      for (int e = 0; e < D; ++e) acc = fmaf(qS[hh * D + e], kb[e], acc);
-      sc = fmaf(acc, a.scale, a.hbias_pages[(size_t)p * a.h + gi * G + hh]);
-    }
-    a.score[((size_t)bi * a.h + gi * G + hh) * K + s] = sc;
-    if (hh == 0) a.idx[((size_t)bi * a.g + gi) * K + s] = c;
-  }
-}
-
-template <typename T, int D, int G>
-static cudaError_t launch_dec_sel(const DecodeSelectArgs& a, cudaStream_t st) {
-  const unsigned blocks = (unsigned)a.b * a.g;
-  if (blocks == 0) return cudaSuccess;
-  decode_select_kernel<T, D, G><<<blocks, kDecSelThreads, 0, st>>>(a);
-  return cudaGetLastError();
-}
-
-template <typename T, int D>
-static cudaError_t dec_sel_by_group(const DecodeSelectArgs& a, cudaStream_t st) {
-  switch (a.h / a.g) {
-    case 1: return launch_dec_sel<T, D, 1>(a, st);
-    case 2: return launch_dec_sel<T, D, 2>(a, st);
-    case 4: return launch_dec_sel<T, D, 4>(a, st);
-    case 8: return launch_dec_sel<T, D, 8>(a, st);
-  }
-  return cudaErrorInvalidValue;
-}
-
-cudaError_t run_decode_select(const DecodeSelectArgs& a, cudaStream_t st) {
-  if (a.bf16) return a.d == 64 ? dec_sel_by_group<__nv_bfloat16, 64>(a, st) : dec_sel_by_group<__nv_bfloat16, 128>(a, st);
-  return a.d == 64 ? dec_sel_by_group<float, 64>(a, st) : dec_sel_by_group<float, 128>(a, st);
 }
 
 }  // namespace hils

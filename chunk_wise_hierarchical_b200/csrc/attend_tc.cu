@@ -5,20 +5,38 @@
 //
 // Work decomposition ("row owner, chunk buckets").  One CTA owns a block of QB
 // consecutive queries of one (sequence, KV head) and all G query heads of the
-// group: R = QB*G rows whose fp32 output accumulators stay in shared memory for
-// the whole CTA.  The CTA buckets its rows' selections by chunk (counting sort
-// in shared memory), then walks the chunks in index order.  For chunk c the
-// rows that selected it are gathered into 128-row tiles:
+// group: R = QB*G rows whose fp32 output accumulators stay in shared memory
+// for the whole CTA.  The CTA buckets its rows' selections by chunk (counting
+// sort in shared memory) and turns them into a list of work items: 128-row
+// tiles of (own chunk | selected chunk c, rows).  Per item
 //     S = Q_tile K_c^T          (tcgen05, M=128 N=64, S in TMEM)
-//     P'_j = exp(x_j - m) * alpha / l,  alpha = exp(shat - M) / Z'   (registers)
-//     O_tile = P' V_c           (tcgen05, M=128 N=d, TMEM)
-//     O[row] += O_tile[row]     (shared memory)
-// so every (row, chunk) pair contributes its already-weighted term and no
-// partial result leaves the SM.  The own causal chunk is processed first; it
-// fixes LSE_own and with it the fusion max M and normaliser Z' of each row.
+//     P_j = exp(x_j - m)        (registers -> bf16 shared memory)
+//     O_tile = P V_c            (tcgen05, M=128 N=d, TMEM)
+//     O[row] (=|+=) f * O_tile[row]   (shared memory)
+// so every (row, chunk) pair contributes its final weighted term and no
+// partial result leaves the SM.  For a selected chunk f = exp(shat - M)/(Z' l);
+// for the own chunk f = exp(m - M)/Z', where the own item completes the
+// fusion max M and normaliser Z' from LSE_own = m + log l.  Own items run first.
+//
+// Warp roles (512 threads), synchronised by mbarriers with bounded waits:
+//   warp 0      producer: cp.async gather of the tile's Q rows (completed, fenced
+//               for the async proxy, then signalled) and a TMA load of K_c into a
+//               ring of operand stages; a stage's Q/K half is reused once S has run
+//   warp 1      producer (one thread): TMA load of V_c, released after P.V
+//   warp 2      MMA issuer (one thread): an event loop issuing S(i) and P.V(j)
+//               as their inputs become ready; tcgen05.commit signals the rest
+//   warps 4-11  two softmax warpgroups taking alternate items: TMEM ->
+//               registers -> P = exp(x - m) (bf16, swizzled smem) and the row's
+//               output multiplier
+//   warps 12-15 epilogue warpgroup: TMEM -> O_tile * multiplier -> shared-memory
+//               accumulators
 // Rows outside a tile's count are computed and ignored (padding of the
 // 128-row MMA).  Summation over chunks runs in chunk-index order, so results
 // do not depend on the order of rows inside a bucket.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_util.cuh"
@@ -27,36 +45,45 @@ namespace hils {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kOwnFlag = 0x80000000u;
+
+template <int D>
+struct TcCfg {
+  static constexpr int NS = D == 64 ? 2 : 1;         // operand stages
+  static constexpr int NP = D == 64 ? 2 : 1;         // S (TMEM) / P (smem) slots
+  static constexpr int kRows = D == 64 ? 384 : 256;  // target rows (QB * G) per CTA
+  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
+  static constexpr uint32_t kStageA = 128 * D * 2, kStageK = 64 * D * 2, kStageV = 64 * D * 2;
+  static constexpr uint32_t kStage = kStageA + kStageK + kStageV;
+  static constexpr uint32_t kStageStride = (kStage + 1023) / 1024 * 1024;
+};
 
 struct TcSmem {
-  uint32_t a, k, v, p;       // byte offsets of the swizzled operand tiles
-  uint32_t o;                // fp32 accumulators [R][D] (float4 XOR-swizzled by row)
-  uint32_t list;             // u16 bucket entries
-  uint32_t off;              // int offsets [n_cand + 1]
-  uint32_t cur;              // int cursors [n_cand]
-  uint32_t rowm, rowz;       // per row: fusion max M and 1/Z'
-  uint32_t tile;             // per tile row: r | slot << 16
-  uint32_t total;
+  uint32_t stage, p, o, list, off, items, rowm, rowz, total;
 };
 
 __host__ __device__ inline uint32_t align_to(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline TcSmem tc_layout(int D, int G, int qb, int K, int n_cand) {
+__host__ __device__ inline int max_items(int G, int qb, int K, int n_cand) {
+  const int own_tiles = (qb / 64 + 2) * ((64 * G + 127) / 128);
+  return own_tiles + n_cand + (qb * K * G + 127) / 128 + 1;
+}
+
+template <int D>
+__host__ __device__ inline TcSmem tc_layout(int G, int qb, int K, int n_cand) {
+  using C = TcCfg<D>;
   TcSmem L;
   uint32_t off = 0;
-  L.a = off; off += 128 * D * 2;
-  L.k = off; off += 64 * D * 2;
-  L.v = off; off += 64 * D * 2;
-  L.p = off; off += 128 * 64 * 2;
+  L.stage = off; off += C::NS * C::kStageStride;
+  L.p = off; off += C::NP * 128 * 64 * 2;
   L.o = off; off += (uint32_t)qb * G * D * 4;
   L.list = off; off = align_to(off + (uint32_t)qb * K * 2, 16);
-  L.off = off; off += (uint32_t)(n_cand + 1) * 4;
-  L.cur = off; off = align_to(off + (uint32_t)n_cand * 4, 16);
+  L.off = off; off = align_to(off + (uint32_t)(2 * n_cand + 2) * 4, 16);
+  L.items = off; off = align_to(off + (uint32_t)max_items(G, qb, K, n_cand) * 4, 16);
   L.rowm = off; off += (uint32_t)qb * G * 4;
   L.rowz = off; off += (uint32_t)qb * G * 4;
-  L.tile = off; off += 128 * 4;
   L.total = align_to(off, 16);
   return L;
 }
@@ -66,17 +93,69 @@ __device__ __forceinline__ float4* o_row_f4(unsigned char* base, uint32_t o_off,
   return reinterpret_cast<float4*>(base + o_off + (size_t)r * D * 4 + (size_t)((j4 ^ (r & 7)) * 16));
 }
 
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+
+// Exclusive scan of v[0..n) in place over the whole block; returns the total.
+__device__ int block_exclusive_scan(int* v, int n, int* wsum) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int seg = (n + kThreads - 1) / kThreads;
+  const int lo = min(tid * seg, n), hi = min(lo + seg, n);
+  int sum = 0;
+  for (int c = lo; c < hi; ++c) sum += v[c];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int wbase = 0, total = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) wbase += wsum[w];
+    total += wsum[w];
+  }
+  int run = wbase + incl - sum;
+  for (int c = lo; c < hi; ++c) {
+    const int x = v[c];
+    v[c] = run;
+    run += x;
+  }
+  __syncthreads();
+  return total;
+}
+
 }  // namespace
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(TcAttendArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ TcAttendArgs a) {
+  using C = TcCfg<D>;
+  constexpr int NS = C::NS, NP = C::NP;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t bars[2];
+  // stage ring: Q tile + K chunk (full_qk) and V chunk (full_v).  A stage's Q/K half is
+  // free once S of its item completed (sfull), its V half once P.V completed (ofull):
+  // each MMA group is committed to exactly one barrier, which every consumer waits on
+  static_assert(NS == NP, "stage and S-slot rings must have the same depth");
+  __shared__ uint64_t bar_full_qk[NS], bar_full_v[NS];
+  __shared__ uint64_t bar_sfull[NP], bar_pfull[NP], bar_ofull[2], bar_ofree[2];
+  __shared__ uint64_t bar_mfull[4];  // the item's row multipliers are written (ring of 4 items)
   __shared__ uint32_t tmem_base_s;
+  __shared__ int s_wsum[kThreads / 32];
+  __shared__ int s_n_items;
+  __shared__ volatile int s_abort;
+  __shared__ float s_mult[4][128];  // per item (ring of 4) and tile row: epilogue multiplier
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = a.n, K = a.top_k, QB = a.qb;
   const int nqb = (N + QB - 1) / QB;
   const int blk = blockIdx.x % nqb;
@@ -85,331 +164,495 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(TcAttendArgs a) 
   const int q0 = blk * QB;
   const int nq = min(QB, N - q0);
   const int head0 = gi * G;
-  const int n_cand = min((q0 + nq - 1) / kChunk, N / kChunk);  // chunks any row of the block may select
-  const TcSmem L = tc_layout(D, G, QB, K, a.n_cand_max);
-  constexpr uint32_t kTmemCols = D == 64 ? 128 : 256;
+  const int n_cand = min((q0 + nq - 1) / kChunk, N / kChunk);
+  const TcSmem L = tc_layout<D>(G, QB, K, a.n_cand_max);
 
   uint16_t* s_list = reinterpret_cast<uint16_t*>(sm + L.list);
-  int* s_off = reinterpret_cast<int*>(sm + L.off);
-  int* s_cur = reinterpret_cast<int*>(sm + L.cur);
+  int* s_off = reinterpret_cast<int*>(sm + L.off);          // [n_cand + 1] bucket offsets
+  int* s_toff = s_off + (a.n_cand_max + 1);                 // [n_cand] item offsets
+  uint32_t* s_items = reinterpret_cast<uint32_t*>(sm + L.items);
   float* s_rowm = reinterpret_cast<float*>(sm + L.rowm);
   float* s_rowz = reinterpret_cast<float*>(sm + L.rowz);
-  uint32_t* s_tile = reinterpret_cast<uint32_t*>(sm + L.tile);
-  const uint32_t sA = tc::smem_u32(sm + L.a), sK = tc::smem_u32(sm + L.k), sV = tc::smem_u32(sm + L.v),
-                 sP = tc::smem_u32(sm + L.p);
-  const uint32_t barS = tc::smem_u32(&bars[0]), barO = tc::smem_u32(&bars[1]);
 
-  const __nv_bfloat16* qg = a.q + ((size_t)bi * a.h + head0) * N * D;       // head0 rows
+  const __nv_bfloat16* qg = a.q + ((size_t)bi * a.h + head0) * N * D;
   const __nv_bfloat16* kg = a.k + ((size_t)bi * a.g + gi) * N * D;
   const __nv_bfloat16* vg = a.v + ((size_t)bi * a.g + gi) * N * D;
   const int32_t* idxg = a.idx + ((size_t)bi * a.g + gi) * N * K;
   const float* sselg = a.ssel + ((size_t)bi * a.h + head0) * N * K;
 
   if (tid == 0) {
-    tc::mbar_init(barS, 1);
-    tc::mbar_init(barO, 1);
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(tc::smem_u32(&bar_full_qk[s]), 32 + 1);  // 32 producer lanes + K's expect_tx
+      tc::mbar_init(tc::smem_u32(&bar_full_v[s]), 1);
+    }
+    for (int s = 0; s < NP; ++s) {
+      tc::mbar_init(tc::smem_u32(&bar_sfull[s]), 1);
+      tc::mbar_init(tc::smem_u32(&bar_pfull[s]), 128);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(tc::smem_u32(&bar_ofull[s]), 1);
+      tc::mbar_init(tc::smem_u32(&bar_ofree[s]), 128);
+    }
+    for (int s = 0; s < 4; ++s) tc::mbar_init(tc::smem_u32(&bar_mfull[s]), 128);
     tc::mbar_fence_init();
+    s_abort = 0;
   }
-  if (warp == 0) tc::tmem_alloc(tc::smem_u32(&tmem_base_s), kTmemCols);
+  if (warp == 0) tc::tmem_alloc(tc::smem_u32(&tmem_base_s), C::kTmemCols);
 
-  // ---- bucket the block's selections by chunk (counting sort) ----
+  // ---------------- buckets and work items ----------------
   for (int c = tid; c <= n_cand; c += kThreads) s_off[c] = 0;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base_s;
-  const uint32_t tS = tmem, tO = tmem + 64;
-  const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-
-  for (int e = tid; e < nq * K; e += kThreads) {
-    const int qo = e / K, i = q0 + qo;
-    const int c = idxg[(size_t)i * K + (e % K)];
-    if (c < 0) continue;
-    if (c >= i / kChunk) { set_error(a.err, kErrBadPage); continue; }
-    atomicAdd(&s_off[c], 1);
-  }
-  __syncthreads();
-  {  // exclusive scan of s_off[0..n_cand) in place, s_off[n_cand] = total
-    const int seg = (n_cand + kThreads - 1) / kThreads;
-    const int lo = min(tid * seg, n_cand), hi = min(lo + seg, n_cand);
-    int sum = 0;
-    for (int c = lo; c < hi; ++c) sum += s_off[c];
-    // block-wide exclusive scan of the per-thread sums
-    int incl = sum;
-    const int lane = tid & 31;
+  // this CTA's selections are contiguous in idx: [q0*K, (q0+nq)*K); loads are issued in
+  // batches before the shared-memory atomics so their latencies overlap
+  constexpr int kLB = 8;
+  const int n_sel_all = nq * K;
+  const int32_t* idx_blk = idxg + (size_t)q0 * K;
+  for (int e0 = tid; e0 < n_sel_all; e0 += kThreads * kLB) {
+    int cv[kLB];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+    for (int u = 0; u < kLB; ++u) {
+      const int e = e0 + u * kThreads;
+      cv[u] = e < n_sel_all ? __ldg(idx_blk + e) : -1;
     }
-    __shared__ int wsum[kThreads / 32];
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int wbase = 0;
-    for (int w = 0; w < warp; ++w) wbase += wsum[w];
-    int run = wbase + incl - sum;
-    __syncthreads();
-    for (int c = lo; c < hi; ++c) {
-      const int x = s_off[c];
-      s_off[c] = run;
-      s_cur[c] = run;
-      run += x;
+#pragma unroll
+    for (int u = 0; u < kLB; ++u) {
+      const int e = e0 + u * kThreads;
+      const int c = cv[u];
+      if (c < 0) continue;
+      if (c >= (q0 + e / K) / kChunk) { set_error(a.err, kErrBadPage); continue; }
+      atomicAdd(&s_off[c], 1);
     }
-    if (tid == kThreads - 1) s_off[n_cand] = wbase + incl;
   }
   __syncthreads();
-  for (int e = tid; e < nq * K; e += kThreads) {
-    const int qo = e / K, s = e % K, i = q0 + qo;
-    const int c = idxg[(size_t)i * K + s];
-    if (c < 0 || c >= i / kChunk) continue;
-    const int pos = atomicAdd(&s_cur[c], 1);
-    s_list[pos] = (uint16_t)(qo | (s << 9));
+  for (int c = tid; c < n_cand; c += kThreads) s_toff[c] = (s_off[c] * G + 127) / 128;  // tiles per chunk
+  __syncthreads();
+  const int n_entries = block_exclusive_scan(s_off, n_cand, s_wsum);
+  const int n_sel_items = block_exclusive_scan(s_toff, n_cand, s_wsum);
+  // cursors for the scatter: a copy of the offsets in the per-row array (rows > n_cand)
+  int* cur = reinterpret_cast<int*>(s_rowm);
+  for (int c = tid; c < n_cand; c += kThreads) cur[c] = s_off[c];
+  if (tid == 0) s_off[n_cand] = n_entries;
+  __syncthreads();
+  for (int e0 = tid; e0 < n_sel_all; e0 += kThreads * kLB) {
+    int cv[kLB];
+#pragma unroll
+    for (int u = 0; u < kLB; ++u) {
+      const int e = e0 + u * kThreads;
+      cv[u] = e < n_sel_all ? __ldg(idx_blk + e) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kLB; ++u) {
+      const int e = e0 + u * kThreads;
+      const int c = cv[u];
+      const int qo = e / K;
+      if (c < 0 || c >= (q0 + qo) / kChunk) continue;
+      const int pos = atomicAdd(&cur[c], 1);
+      s_list[pos] = (uint16_t)(qo | ((e % K) << 9));
+    }
   }
+  // items: the own chunks' tiles first, then every selected chunk's tiles
+  const int oc_first = q0 / kChunk, oc_last = (q0 + nq - 1) / kChunk;
+  if (tid == 0) {
+    int n = 0;
+    for (int oc = oc_first; oc <= oc_last; ++oc) {
+      const int qa = max(q0, oc * kChunk) - q0, qb = min(q0 + nq, oc * kChunk + kChunk) - q0;
+      for (int t0 = 0; t0 < (qb - qa) * G; t0 += 128) s_items[n++] = kOwnFlag | ((uint32_t)oc << 16) | (uint32_t)t0;
+    }
+    s_n_items = n;
+  }
+  __syncthreads();
+  const int n_own_items = s_n_items;
+  for (int c = tid; c < n_cand; c += kThreads) {
+    const int rows = (s_off[c + 1] - s_off[c]) * G;
+    int base = n_own_items + s_toff[c];
+    for (int t0 = 0; t0 < rows; t0 += 128) s_items[base++] = ((uint32_t)c << 16) | (uint32_t)t0;
+  }
+  const int n_items = n_own_items + n_sel_items;
   __syncthreads();
 
-  uint32_t phase = 0;
-  bool failed = false;
+  // item -> tile geometry
+  auto item_rows = [&](uint32_t it, int& c, bool& own, int& t0, int& n_rows) {
+    own = (it & kOwnFlag) != 0;
+    c = (int)((it >> 16) & 0x7fffu);
+    t0 = (int)(it & 0xffffu);
+    if (own) {
+      const int qa = max(q0, c * kChunk) - q0, qb = min(q0 + nq, c * kChunk + kChunk) - q0;
+      n_rows = min(128, (qb - qa) * G - t0);
+    } else {
+      n_rows = min(128, (s_off[c + 1] - s_off[c]) * G - t0);
+    }
+  };
+  // tile row t of an item -> row r of the block (and the score slot for selected chunks)
+  auto row_of = [&](bool own, int c, int t0, int t, int& r, int& slot) {
+    const int x = t0 + t;
+    if (own) {
+      const int qa = max(q0, c * kChunk) - q0;
+      r = (qa + x / G) * G + x % G;
+      slot = -1;
+    } else {
+      const uint32_t e = s_list[s_off[c] + x / G];
+      r = (int)(e & 511u) * G + x % G;
+      slot = (int)(e >> 9);
+    }
+  };
+  auto stage_ptr = [&](int s) -> unsigned char* { return sm + L.stage + s * C::kStageStride; };
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    const uint32_t b = tc::smem_u32(bar);
+    for (uint32_t it = 0; it < (1u << 26); ++it) {
+      if (tc::mbar_test(b, parity)) return true;
+      if ((it & 1023u) == 1023u && s_abort) return false;
+    }
+    set_error(a.err, kErrTimeout);
+    s_abort = 1;
+    return false;
+  };
   const float sc2 = a.scale * kLog2e;
 
-  // loads one chunk's K and V (rows >= nvalid zero-filled) into the swizzled tiles
-  auto load_kv = [&](int c, int nvalid) {
-    const __nv_bfloat16* kc = kg + (size_t)c * kChunk * D;
-    const __nv_bfloat16* vc = vg + (size_t)c * kChunk * D;
-    constexpr int CH = D / 8;  // 16-byte chunks per row
-    for (int x = tid; x < kChunk * CH; x += kThreads) {
-      const int r = x / CH, ch = x % CH;
-      const uint32_t o = (uint32_t)(ch >> 3) * 8192u + tc::sw128_chunk(r, ch & 7);
-      const bool ok = r < nvalid;
-      const size_t src = ok ? (size_t)r * D + ch * 8 : 0;
-      tc::cp_async16(sK + o, kc + src, ok ? 16 : 0);
-      tc::cp_async16(sV + o, vc + src, ok ? 16 : 0);
-    }
-  };
-  // gathers the Q rows of a tile: row t -> (query offset, head)
-  auto gather_q = [&](int n_rows) {
-    constexpr int CH = D / 8;
-    for (int x = tid; x < n_rows * CH; x += kThreads) {
-      const int t = x / CH, ch = x % CH;
-      const int r = (int)(s_tile[t] & 0xffffu);
-      const int qo = r / G, hh = r % G;
-      const __nv_bfloat16* src = qg + ((size_t)hh * N + q0 + qo) * D + ch * 8;
-      tc::cp_async16(sA + (uint32_t)(ch >> 3) * 16384u + tc::sw128_chunk(t, ch & 7), src);
-    }
-  };
-  // S = Q K^T into TMEM (one thread)
-  auto issue_s = [&]() {
-    constexpr uint32_t id = tc::make_idesc_bf16(128, 64, false, false);
+  if (warp == 0) {
+    // ======================= producer: Q rows (cp.async gather) + K chunk (TMA) =======================
+    // The Q rows are written through the generic proxy: each lane waits for its own
+    // copies, fences them for the tensor core (async proxy), then arrives.  With two
+    // stages one item's copies stay in flight while the next item is issued.
+    auto publish = [&](int j) {  // item j's copies are complete and fenced
+      tc::fence_async_smem();
+      mbar_arrive(tc::smem_u32(&bar_full_qk[j % NS]));
+    };
+    for (int i = 0; i < n_items; ++i) {
+      const int s = i % NS;
+      if (i >= NS && !wait(&bar_sfull[(i - NS) % NP], (uint32_t)(((i - NS) / NP) & 1))) break;
+      int c, t0, n_rows;
+      bool own;
+      item_rows(s_items[i], c, own, t0, n_rows);
+      const uint32_t sA = tc::smem_u32(stage_ptr(s)), sK = sA + C::kStageA;
+      const uint32_t full = tc::smem_u32(&bar_full_qk[s]);
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(full, C::kStageK);
 #pragma unroll
-    for (int k = 0; k < D / 16; ++k) {
-      const uint64_t da = tc::make_desc(sA + (k >> 2) * 16384u + (k & 3) * 32u, 16, 1024);
-      const uint64_t db = tc::make_desc(sK + (k >> 2) * 8192u + (k & 3) * 32u, 16, 1024);
-      tc::mma_bf16(tS, da, db, id, k > 0);
-    }
-    tc::mma_commit(barS);
-  };
-  // O_tile = P V into TMEM (one thread)
-  auto issue_pv = [&]() {
-    constexpr uint32_t id = tc::make_idesc_bf16(128, D, false, true);
+        for (int x = 0; x < D / 64; ++x)
+          tc::tma_load_3d(sK + x * 8192u, &a.tmap_k, x * 64, c * kChunk, bi * a.g + gi, full);
+      }
+      constexpr int CH = D / 8;  // 16-byte pieces per row
+      for (int t = lane; t < n_rows; t += 32) {
+        int r, slot;
+        row_of(own, c, t0, t, r, slot);
+        const __nv_bfloat16* src = qg + ((size_t)(r % G) * N + q0 + r / G) * D;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint64_t da = tc::make_desc(sP + k * 32u, 16, 1024);
-      const uint64_t db = tc::make_desc(sV + k * 2048u, 8192, 1024);
-      tc::mma_bf16(tO, da, db, id, k > 0);
+        for (int ch = 0; ch < CH; ++ch)
+          tc::cp_async16(sA + (uint32_t)(ch >> 3) * 16384u + tc::sw128_chunk(t, ch & 7), src + ch * 8);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if constexpr (NS == 1) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        publish(i);
+      } else {
+        if (i >= 1) {
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+          publish(i - 1);
+        }
+        if (i == n_items - 1) {
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
+          publish(i);
+        }
+      }
+      if (s_abort) break;
     }
-    tc::mma_commit(barO);
-  };
-  // softmax of this thread's tile row (called by whole warps: the TMEM loads are
-  // warp-collective); writes P' = exp(x - m) * f into the P tile when `valid`.
-  // mult_after_l: f = mult / l, else f = mult.  Returns m (log2-domain max) and l.
-  auto softmax_row = [&](int t, bool valid, int jmax, float mult, bool mult_after_l, float& m_out,
-                         float& l_out) {
-    float s[64];
-    tc::tmem_ld32(tS + lane_off, s);
-    tc::tmem_ld32(tS + lane_off + 32, s + 32);
-    tc::tmem_wait_ld();
-    float m = -INFINITY;
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 1) {
+    // ======================= producer: V chunk (TMA) =======================
+    if (lane == 0) {
+      for (int i = 0; i < n_items; ++i) {
+        const int s = i % NS;
+        // P.V of item i - NS must have completed
+        if (i >= NS && !wait(&bar_ofull[(i - NS) & 1], (uint32_t)(((i - NS) >> 1) & 1))) break;
+        const int c = (int)((s_items[i] >> 16) & 0x7fffu);
+        const uint32_t sV = tc::smem_u32(stage_ptr(s)) + C::kStageA + C::kStageK;
+        const uint32_t full = tc::smem_u32(&bar_full_v[s]);
+        tc::mbar_arrive_expect_tx(full, C::kStageV);
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      s[j] = j <= jmax ? s[j] * sc2 : -INFINITY;  // log2 domain
-      m = fmaxf(m, s[j]);
-    }
-    float l = 0.f;
-#pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      s[j] = exp2f(s[j] - m);
-      l += s[j];
-    }
-    const float f = mult_after_l ? mult / l : mult;
-    if (valid) {
-      unsigned char* prow = sm + L.p;
-#pragma unroll
-      for (int j = 0; j < 64; j += 8) {
-        uint4 pk;
-        pk.x = tc::pack_bf16x2(s[j] * f, s[j + 1] * f);
-        pk.y = tc::pack_bf16x2(s[j + 2] * f, s[j + 3] * f);
-        pk.z = tc::pack_bf16x2(s[j + 4] * f, s[j + 5] * f);
-        pk.w = tc::pack_bf16x2(s[j + 6] * f, s[j + 7] * f);
-        *reinterpret_cast<uint4*>(prow + tc::sw128_chunk(t, j >> 3)) = pk;
+        for (int x = 0; x < D / 64; ++x) tc::tma_load_3d(sV + x * 8192u, &a.tmap_v, x * 64, c * kChunk, bi * a.g + gi, full);
       }
     }
-    m_out = m;
-    l_out = l;
-  };
-  // waits for an MMA group; a timeout is recorded and aborts the CTA
-  auto wait_bar = [&](uint32_t bar) {
-    if (!tc::mbar_wait(bar, phase)) {
-      set_error(a.err, kErrTimeout);
-      failed = true;
+  } else if (warp == 2) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      const uint32_t tS0 = tmem, tO0 = tmem + NP * 64;
+      constexpr uint32_t idS = tc::make_idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idO = tc::make_idesc_bf16(128, D, false, true);
+      auto issue_s = [&](int i) {
+        const int s = i % NS, b = i % NP;
+        const uint32_t sA = tc::smem_u32(stage_ptr(s)), sK = sA + C::kStageA;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t da = tc::make_desc(sA + (k >> 2) * 16384u + (k & 3) * 32u, 16, 1024);
+          const uint64_t db = tc::make_desc(sK + (k >> 2) * 8192u + (k & 3) * 32u, 16, 1024);
+          tc::mma_bf16(tS0 + b * 64, da, db, idS, k > 0);
+        }
+        tc::mma_commit(tc::smem_u32(&bar_sfull[b]));
+      };
+      auto issue_pv = [&](int i) {
+        const int s = i % NS, b = i % NP, o = i & 1;
+        const uint32_t sP = tc::smem_u32(sm + L.p + b * 16384);
+        const uint32_t sV = tc::smem_u32(stage_ptr(s)) + C::kStageA + C::kStageK;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t da = tc::make_desc(sP + k * 32u, 16, 1024);
+          const uint64_t db = tc::make_desc(sV + k * 2048u, 8192, 1024);
+          tc::mma_bf16(tO0 + o * D, da, db, idO, k > 0);
+        }
+        tc::mma_commit(tc::smem_u32(&bar_ofull[o]));
+      };
+      // event loop: issue S(next_s) as soon as its operands have landed and its S slot
+      // is free, and P.V(next_pv) as soon as its P is written and its TMEM slot is free
+      int next_s = 0, next_pv = 0;
+      uint32_t idle = 0;
+      while (next_pv < n_items) {
+        bool progressed = false;
+        if (next_s < n_items && next_s < next_pv + NP &&
+            tc::mbar_test(tc::smem_u32(&bar_full_qk[next_s % NS]), (uint32_t)((next_s / NS) & 1))) {
+          tc::fence_after_sync();
+          issue_s(next_s);
+          ++next_s;
+          progressed = true;
+        }
+        if (next_pv < next_s &&
+            tc::mbar_test(tc::smem_u32(&bar_pfull[next_pv % NP]), (uint32_t)((next_pv / NP) & 1)) &&
+            tc::mbar_test(tc::smem_u32(&bar_full_v[next_pv % NS]), (uint32_t)((next_pv / NS) & 1)) &&
+            (next_pv < 2 ||
+             tc::mbar_test(tc::smem_u32(&bar_ofree[next_pv & 1]), (uint32_t)(((next_pv - 2) >> 1) & 1)))) {
+          tc::fence_after_sync();
+          issue_pv(next_pv);
+          ++next_pv;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle >= (1u << 26) || ((idle & 1023u) == 1023u && s_abort)) {
+          if (!s_abort) {
+            set_error(a.err, kErrTimeout);
+            s_abort = 1;
+          }
+          break;
+        }
+      }
     }
-  };
-
-  // ---------------- own (causal) chunks: LSE_own, fusion constants, O init ----------------
-  const int oc_first = q0 / kChunk, oc_last = (q0 + nq - 1) / kChunk;
-  for (int oc = oc_first; oc <= oc_last && !failed; ++oc) {
-    const int qa = max(q0, oc * kChunk) - q0, qb = min(q0 + nq, oc * kChunk + kChunk) - q0;
-    load_kv(oc, min(kChunk, N - oc * kChunk));
-    for (int t0 = qa * G; t0 < qb * G; t0 += 128) {
-      const int n_rows = min(128, qb * G - t0);
-      if (tid < n_rows) s_tile[tid] = (uint32_t)(t0 + tid);
-      __syncthreads();
-      gather_q(n_rows);
-      tc::cp_async_wait_all();
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      if (tid == 0) issue_s();
-      wait_bar(barS);
-      if (__syncthreads_or(failed)) { failed = true; break; }
-      tc::fence_after_sync();
-      float m = 0.f, l = 1.f;
-      const bool row_ok = tid < n_rows;
-      const bool warp_ok = warp * 32 < n_rows;
-      const int r = row_ok ? t0 + tid : 0;
+  } else if (warp >= 4 && warp < 12) {
+    // ======================= softmax (two warpgroups, alternating items) =======================
+    const int wg = (warp - 4) >> 2;      // warpgroup: handles items i with i % NP == wg
+    const int t = (tid - 128) & 127;     // tile row == TMEM lane
+    const int wq = warp & 3;             // TMEM lane quadrant
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    // per-row fusion terms of the selected chunks: Mx = max shat, Zx = sum exp(shat - Mx);
+    // the own item turns them into (M, 1/Z') with LSE_own
+    for (int r = tid - 128; r < nq * G; r += 256) {
       const int qo = r / G, hh = r % G, i = q0 + qo;
-      if (warp_ok) softmax_row(tid, row_ok, row_ok ? i - oc * kChunk : 63, 1.0f, false, m, l);
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      if (tid == 0) issue_pv();
-      wait_bar(barO);
-      if (__syncthreads_or(failed)) { failed = true; break; }
-      tc::fence_after_sync();
-      if (warp_ok) {
-        // m, l are in the log2 domain: LSE_own = (m + log2 l) / log2(e)
-        const float lse = (m + log2f(l)) / kLog2e;
-        float M = lse;
-        const int32_t* ir = idxg + (size_t)i * K;
-        const float* sr = sselg + ((size_t)hh * N + i) * K;
-        const int kk = row_ok ? K : 0;
-        for (int s = 0; s < kk; ++s) {
-          const int c = ir[s];
-          if (c >= 0 && c < i / kChunk) M = fmaxf(M, sr[s]);
-        }
-        float Z = expf(lse - M);
-        for (int s = 0; s < kk; ++s) {
-          const int c = ir[s];
-          if (c >= 0 && c < i / kChunk) Z += expf(sr[s] - M);
-        }
-        if (row_ok) {
-          s_rowm[r] = M;
-          s_rowz[r] = 1.0f / Z;
-        }
-        // own term: exp(LSE_own - M)/Z' * (sum_j p_j v_j)/l = exp(m_nat - M)/Z' * sum_j p_j v_j
-        const float w = expf(m / kLog2e - M) / Z;
+      const int32_t* ir = idxg + (size_t)i * K;
+      const float* sr = sselg + ((size_t)hh * N + i) * K;
+      float mx = -INFINITY, zx = 0.f;  // online max / shifted sum over the valid slots
+      for (int s0 = 0; s0 < K; s0 += 8) {
+        float v[8];
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tc::tmem_ld32(tO + lane_off + c0, o);
-          tc::tmem_wait_ld();
-          if (row_ok) {
+        for (int u = 0; u < 8; ++u) {
+          const int s = s0 + u;
+          const int c = s < K ? __ldg(ir + s) : -1;
+          const float x = s < K ? __ldg(sr + s) : -INFINITY;
+          v[u] = (c >= 0 && c < i / kChunk) ? x : -INFINITY;
+        }
+        float bm = v[0];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *o_row_f4(sm, L.o, r, (c0 + j) >> 2, D) =
-                  make_float4(o[j] * w, o[j + 1] * w, o[j + 2] * w, o[j + 3] * w);
+        for (int u = 1; u < 8; ++u) bm = fmaxf(bm, v[u]);
+        if (bm == -INFINITY) continue;
+        const float nm = fmaxf(mx, bm);
+        float add = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) add += expf(v[u] - nm);
+        zx = zx * expf(mx - nm) + add;
+        mx = nm;
+      }
+      s_rowm[r] = mx;
+      s_rowz[r] = zx;
+    }
+    named_bar(1, 256);
+    // score of this thread's row in item i (selected chunks only), loaded one item ahead
+    auto row_score = [&](int i) -> float {
+      if (i >= n_items) return 0.f;
+      int c, t0, n_rows;
+      bool own;
+      item_rows(s_items[i], c, own, t0, n_rows);
+      if (own || t >= n_rows) return 0.f;
+      int r, slot;
+      row_of(own, c, t0, t, r, slot);
+      return __ldg(sselg + ((size_t)(r % G) * N + q0 + r / G) * K + slot);
+    };
+    float sh_next = row_score(wg);
+    bool synced_own = false;
+    for (int i = wg; i < n_items && wg < NP; i += NP) {
+      const int b = i % NP;
+      bool ok_loop = true;
+      int c, t0, n_rows;
+      bool own;
+      item_rows(s_items[i], c, own, t0, n_rows);
+      const float sh = sh_next;
+      sh_next = row_score(i + NP);
+      if (!own && !synced_own) {
+        named_bar(1, 256);  // every row's (M, 1/Z') is final once the own items are done
+        synced_own = true;
+      }
+      if (!wait(&bar_sfull[b], (uint32_t)((i / NP) & 1))) break;
+      tc::fence_after_sync();
+      const bool row_ok = t < n_rows;
+      if (wq * 32 < n_rows) {
+        int r = 0, slot = -1;
+        if (row_ok) row_of(own, c, t0, t, r, slot);
+        float s[64];
+        tc::tmem_ld32(tmem + b * 64 + lane_off, s);
+        tc::tmem_ld32(tmem + b * 64 + 32 + lane_off, s + 32);
+        tc::tmem_wait_ld();
+        float mult;  // applied by the epilogue: O_tile row * mult
+        if (!own && sc2 > 0.f) {
+          // lean path (all 64 keys valid): raw max, p = exp2(S*c - m*c), one FFMA + ex2 each
+          float mp[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mp[u] = s[u];
+#pragma unroll
+          for (int j = 8; j < 64; ++j) mp[j & 7] = fmaxf(mp[j & 7], s[j]);
+          const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                 fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          const float moff = mr * sc2;  // scale > 0: the max of the scaled logits
+          float lp[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) lp[u] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            s[j] = exp2f(fmaf(s[j], sc2, -moff));
+            lp[j & 7] += s[j];
+          }
+          const float l = ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+          mult = row_ok ? expf(sh - s_rowm[r]) * s_rowz[r] / l : 0.f;
+        } else {
+          // general path (own chunk: causal mask; LSE_own completes the fusion max and normaliser)
+          const int jmax = (own && row_ok) ? (q0 + r / G) - c * kChunk : 63;
+          float mp[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mp[u] = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            s[j] = j <= jmax ? s[j] * sc2 : -INFINITY;  // log2 domain
+            mp[j & 7] = fmaxf(mp[j & 7], s[j]);
+          }
+          const float m = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          float lp[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) lp[u] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            s[j] = exp2f(s[j] - m);
+            lp[j & 7] += s[j];
+          }
+          const float l = ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+          mult = 0.f;
+          if (row_ok && own) {
+            const float lse = (m + log2f(l)) / kLog2e;  // natural-log LSE_own
+            const float mx = s_rowm[r], zx = s_rowz[r];
+            const float M = fmaxf(lse, mx);
+            const float Z = expf(lse - M) + (zx > 0.f ? zx * expf(mx - M) : 0.f);
+            s_rowm[r] = M;
+            s_rowz[r] = 1.0f / Z;
+            mult = expf(m / kLog2e - M) / Z;
+          } else if (row_ok) {
+            mult = expf(sh - s_rowm[r]) * s_rowz[r] / l;
+          }
+        }
+        // P slot b was last read by P.V(i - NP): it must have completed before it is
+        // overwritten (S(i) completing does not imply it)
+        if (i >= NP && !wait(&bar_ofull[(i - NP) & 1], (uint32_t)(((i - NP) >> 1) & 1))) {
+          ok_loop = false;
+        }
+        if (row_ok && ok_loop) {
+          s_mult[i & 3][t] = mult;
+          unsigned char* prow = sm + L.p + b * 16384;
+#pragma unroll
+          for (int j = 0; j < 64; j += 8) {
+            uint4 pk;
+            pk.x = tc::pack_bf16x2(s[j], s[j + 1]);
+            pk.y = tc::pack_bf16x2(s[j + 2], s[j + 3]);
+            pk.z = tc::pack_bf16x2(s[j + 4], s[j + 5]);
+            pk.w = tc::pack_bf16x2(s[j + 6], s[j + 7]);
+            *reinterpret_cast<uint4*>(prow + tc::sw128_chunk(t, j >> 3)) = pk;
           }
         }
       }
+      tc::fence_async_smem();
       tc::fence_before_sync();
-      __syncthreads();
-      phase ^= 1u;
+      mbar_arrive(tc::smem_u32(&bar_pfull[b]));
+      // the epilogue of item i reads s_mult[i & 3]; it cannot lap this ring: item i + 4
+      // needs S(i+4), which waits for P.V(i+2), which waits for that epilogue
+      mbar_arrive(tc::smem_u32(&bar_mfull[i & 3]));
+      if (!ok_loop) break;
     }
-  }
-
-  // ---------------- selected chunks ----------------
-  for (int c = 0; c < n_cand && !failed; ++c) {
-    const int base = s_off[c], cnt = s_off[c + 1] - base;
-    if (cnt == 0) continue;
-    load_kv(c, kChunk);
-    const int total = cnt * G;
-    for (int t0 = 0; t0 < total; t0 += 128) {
-      const int n_rows = min(128, total - t0);
-      if (tid < n_rows) {
-        const int x = t0 + tid;
-        const uint32_t e = s_list[base + x / G];
-        const int qo = (int)(e & 511u), s = (int)(e >> 9);
-        s_tile[tid] = (uint32_t)(qo * G + x % G) | ((uint32_t)s << 16);
-      }
-      __syncthreads();
-      gather_q(n_rows);
-      tc::cp_async_wait_all();
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      __syncthreads();
+    if (!synced_own) named_bar(1, 256);
+  } else if (warp >= 12) {
+    // ======================= epilogue =======================
+    const int t = tid - 384;
+    const int wq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    const uint32_t tO0 = tmem + NP * 64;
+    for (int i = 0; i < n_items; ++i) {
+      const int o = i & 1;
+      int c, t0, n_rows;
+      bool own;
+      item_rows(s_items[i], c, own, t0, n_rows);
+      if (!wait(&bar_ofull[o], (uint32_t)((i >> 1) & 1))) break;
+      if (!wait(&bar_mfull[i & 3], (uint32_t)((i >> 2) & 1))) break;
       tc::fence_after_sync();
-      if (tid == 0) issue_s();
-      wait_bar(barS);
-      if (__syncthreads_or(failed)) { failed = true; break; }
-      tc::fence_after_sync();
-      int r = 0;
-      const bool row_ok = tid < n_rows;
-      const bool warp_ok = warp * 32 < n_rows;
-      if (warp_ok) {
-        float alpha = 0.f;
+      if (wq * 32 < n_rows) {
+        const bool row_ok = t < n_rows;
+        int r = 0, slot;
+        float mult = 0.f;
         if (row_ok) {
-          const uint32_t e = s_tile[tid];
-          r = (int)(e & 0xffffu);
-          const int s = (int)(e >> 16), qo = r / G, hh = r % G;
-          const float sh = sselg[((size_t)hh * N + q0 + qo) * K + s];
-          alpha = expf(sh - s_rowm[r]) * s_rowz[r];
+          row_of(own, c, t0, t, r, slot);
+          mult = s_mult[i & 3][t];
         }
-        float m, l;
-        softmax_row(tid, row_ok, 63, alpha, true, m, l);
-      }
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      __syncthreads();
-      tc::fence_after_sync();
-      if (tid == 0) issue_pv();
-      wait_bar(barO);
-      if (__syncthreads_or(failed)) { failed = true; break; }
-      tc::fence_after_sync();
-      if (warp_ok) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tc::tmem_ld32(tO + lane_off + c0, o);
+          float v[32];
+          tc::tmem_ld32(tO0 + o * D + c0 + lane_off, v);
           tc::tmem_wait_ld();
           if (row_ok) {
+            float4 u[8];
+            if (!own) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              float4* p = o_row_f4(sm, L.o, r, (c0 + j) >> 2, D);
-              float4 v = *p;
-              v.x += o[j]; v.y += o[j + 1]; v.z += o[j + 2]; v.w += o[j + 3];
-              *p = v;
+              for (int j = 0; j < 8; ++j) u[j] = *o_row_f4(sm, L.o, r, (c0 >> 2) + j, D);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) u[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              u[j].x = fmaf(v[4 * j], mult, u[j].x);
+              u[j].y = fmaf(v[4 * j + 1], mult, u[j].y);
+              u[j].z = fmaf(v[4 * j + 2], mult, u[j].z);
+              u[j].w = fmaf(v[4 * j + 3], mult, u[j].w);
+              *o_row_f4(sm, L.o, r, (c0 >> 2) + j, D) = u[j];
             }
           }
         }
       }
       tc::fence_before_sync();
-      __syncthreads();
-      phase ^= 1u;
+      mbar_arrive(tc::smem_u32(&bar_ofree[o]));
+      // a row sits at different tile positions in different items: finish this item's
+      // read-modify-writes before any epilogue warp starts the next one
+      named_bar(2, 128);
     }
   }
 
   // ---------------- write the block's rows ----------------
-  if (!failed) {
+  tc::fence_before_sync();
+  __syncthreads();
+  if (!s_abort) {
     for (int x = tid; x < nq * G * (D / 4); x += kThreads) {
       const int r = x / (D / 4), j4 = x % (D / 4);
       const int qo = r / G, hh = r % G;
@@ -420,40 +663,70 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(TcAttendArgs a) 
       *reinterpret_cast<uint2*>(a.out + (((size_t)bi * a.h + head0 + hh) * N + q0 + qo) * D + j4 * 4) = pk;
     }
   }
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A [b*g][N][D] bf16 tensor as a rank-3 map with 64 x 64 boxes in the 128-byte
+// swizzle of the MMA operand tiles; rows past N read as zeros.
+static bool encode_kv_map(CUtensorMap* m, const void* base, int D, int N, int bg) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)bg};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Queries per CTA for a shape, or 0 when the shared-memory plan does not fit.
-static int pick_qb(int D, int G, int K, int N, size_t* smem_out) {
-  const int rows_target = D == 64 ? 512 : 256;
-  int qb = rows_target / G;
+template <int D>
+static int pick_qb(int G, int K, int N, size_t* smem_out) {
+  int qb = TcCfg<D>::kRows / G;
   const int n_cand_max = N / kChunk;
-  while (qb >= 16) {
-    const TcSmem L = tc_layout(D, G, qb, K, n_cand_max);
+  for (; qb >= 16; qb >>= 1) {
+    if (qb * G < n_cand_max + 1) continue;  // the scatter cursors borrow the per-row array
+    const TcSmem L = tc_layout<D>(G, qb, K, n_cand_max);
     const size_t need = (size_t)L.total + 1024;
-    if (need <= 227 * 1024 - 512) {  // leave room for the static shared variables
+    if (need <= 227 * 1024 - 1024) {  // leave room for the static shared variables
       *smem_out = need;
       return qb;
     }
-    qb >>= 1;
   }
   return 0;
 }
 
 bool attend_tc_supported(int d, int G, int K, int N) {
   size_t smem;
-  return (d == 64 || d == 128) && K <= 64 && pick_qb(d, G, K, N, &smem) > 0;
+  if (K > 64 || N / kChunk > 32767 || tensor_map_encoder() == nullptr) return false;
+  return d == 64 ? pick_qb<64>(G, K, N, &smem) > 0 : d == 128 ? pick_qb<128>(G, K, N, &smem) > 0 : false;
 }
 
 template <int D, int G>
 static cudaError_t launch_tc(TcAttendArgs a, cudaStream_t st) {
   size_t smem = 0;
-  const int qb = pick_qb(D, G, a.top_k, a.n, &smem);
+  const int qb = pick_qb<D>(G, a.top_k, a.n, &smem);
   if (qb == 0) return cudaErrorInvalidConfiguration;
   a.qb = qb;
   a.n_cand_max = a.n / kChunk;
+  if (!encode_kv_map(&a.tmap_k, a.k, D, a.n, a.b * a.g) || !encode_kv_map(&a.tmap_v, a.v, D, a.n, a.b * a.g))
+    return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

@@ -56,15 +56,21 @@ AttendLayout attend_layout(const hils_shape* s) {
 }
 
 struct DecodeLayout {
-  size_t keys, idx, ssel, total;
+  size_t part_keys, part_att, scan_ticket, att_ticket, idx, sel_page, ssel, total;
 };
 DecodeLayout decode_layout(const hils_shape* s) {
-  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k;
-  const size_t cmax = (s->seq_len + s->chunk - 1) / s->chunk;
+  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k, d = s->head_dim;
+  const size_t G = h / g;
+  const int cmax = (s->seq_len + s->chunk - 1) / s->chunk;
+  const size_t nsplit = hils::decode_splits(cmax);
   DecodeLayout L;
   size_t off = kHeader;
-  L.keys = off; off = align_up(off + b * g * cmax * 8);
+  L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
+  L.part_att = off; off = align_up(off + b * g * (K + 1) * G * (d + 2) * 4);
+  L.scan_ticket = off; off = align_up(off + b * g * 4);
+  L.att_ticket = off; off = align_up(off + b * g * 4);
   L.idx = off; off = align_up(off + b * g * K * 4);
+  L.sel_page = off; off = align_up(off + b * g * K * 4);
   L.ssel = off; off = align_up(off + b * h * K * 4);
   L.total = off;
   return L;
@@ -251,25 +257,21 @@ hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages,
   char* w = static_cast<char*>(ws);
   unsigned* err = reinterpret_cast<unsigned*>(w);
   int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
-  float* ssel = reinterpret_cast<float*>(w + L.ssel);
-  const bool bf16 = s->dtype == HILS_BF16;
-  const float scale = eff_scale(s);
-
-  hils::DecodeSelectArgs ds{};
-  ds.q = q; ds.kbar_pages = kbar_pages; ds.hbias_pages = hbias_pages; ds.block_table = block_table;
-  ds.seq_lens = seq_lens; ds.keys = reinterpret_cast<unsigned long long*>(w + L.keys);
-  ds.idx = idx; ds.score = ssel; ds.err = err;
-  ds.b = s->batch; ds.h = s->heads_q; ds.g = s->heads_kv; ds.d = s->head_dim;
-  ds.max_chunks = max_chunks; ds.top_k = s->top_k; ds.n_pages = n_pages; ds.scale = scale; ds.bf16 = bf16;
-  if (s->top_k > 0 && hils::run_decode_select(ds, cs) != cudaSuccess) return HILS_ERR_CUDA;
-
-  hils::AttendRowsArgs ar{};
-  ar.q = q; ar.k = k_pages; ar.v = v_pages; ar.idx = idx; ar.ssel = ssel; ar.out = out;
-  ar.block_table = block_table; ar.seq_lens = seq_lens; ar.err = err;
-  ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = 1; ar.d = s->head_dim;
-  ar.top_k = s->top_k; ar.max_chunks = max_chunks; ar.n_pages = n_pages; ar.scale = scale;
-  ar.bf16 = bf16; ar.paged = true;
-  return cuda_status(hils::run_attend_rows(ar, cs));
+  hils::DecodeArgs da{};
+  da.q = q; da.k_pages = k_pages; da.v_pages = v_pages; da.kbar_pages = kbar_pages;
+  da.hbias_pages = hbias_pages; da.block_table = block_table; da.seq_lens = seq_lens; da.out = out;
+  da.idx = idx;
+  da.ssel = reinterpret_cast<float*>(w + L.ssel);
+  da.sel_page = reinterpret_cast<int32_t*>(w + L.sel_page);
+  da.part_keys = reinterpret_cast<unsigned long long*>(w + L.part_keys);
+  da.part_att = reinterpret_cast<float*>(w + L.part_att);
+  da.scan_ticket = reinterpret_cast<unsigned*>(w + L.scan_ticket);
+  da.att_ticket = reinterpret_cast<unsigned*>(w + L.att_ticket);
+  da.err = err;
+  da.b = s->batch; da.h = s->heads_q; da.g = s->heads_kv; da.d = s->head_dim; da.top_k = s->top_k;
+  da.max_chunks = max_chunks; da.n_pages = n_pages; da.scale = eff_scale(s);
+  da.bf16 = s->dtype == HILS_BF16;
+  return cuda_status(hils::run_decode(da, cs));
 }
 
 hils_status hils_device_status(void* ws, void* stream) {

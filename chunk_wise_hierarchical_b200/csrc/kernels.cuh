@@ -1,6 +1,7 @@
 // Host-side launch interface of the HiLS kernels (one struct per kernel family).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -33,21 +34,32 @@ struct SelectArgs {
 };
 cudaError_t run_select_simt(const SelectArgs& a, cudaStream_t st);
 
-struct DecodeSelectArgs {
+// Paged decode: split scan + Top-K (last CTA merges), then per-chunk attention
+// with a last-CTA fusion, chained by programmatic dependent launch.
+struct DecodeArgs {
   const void* q;               // [b,h,d]
+  const void* k_pages;         // [P,g,B,d]
+  const void* v_pages;
   const float* kbar_pages;     // [P,h,d]
   const float* hbias_pages;    // [P,h]
   const int32_t* block_table;  // [b,max_chunks]
   const int32_t* seq_lens;     // [b]
-  unsigned long long* keys;    // workspace [b,g,max_chunks]
+  void* out;                   // [b,h,d]
   int32_t* idx;                // [b,g,K]
-  float* score;                // [b,h,K]
+  int32_t* sel_page;           // [b,g,K] page of each selected chunk
+  float* ssel;                 // [b,h,K]
+  unsigned long long* part_keys;  // [b,g,nsplit,K]
+  float* part_att;             // [b,g,K+1,G,d+2]
+  unsigned* scan_ticket;       // [b,g]
+  unsigned* att_ticket;        // [b,g]
   unsigned* err;
-  int b, h, g, d, max_chunks, top_k, n_pages;
+  int b, h, g, d, top_k, max_chunks, n_pages;
+  int nsplit, att_ctas;        // set by the launcher
   float scale;
   bool bf16;
 };
-cudaError_t run_decode_select(const DecodeSelectArgs& a, cudaStream_t st);
+int decode_splits(int max_chunks);
+cudaError_t run_decode(DecodeArgs a, cudaStream_t st);
 
 // Row-wise attention + fusion (one warp per query and KV group).
 struct AttendRowsArgs {
@@ -68,7 +80,9 @@ struct AttendRowsArgs {
 cudaError_t run_attend_rows(const AttendRowsArgs& a, cudaStream_t st);
 
 // Tensor-core prefill attention + fusion for a given selection (bf16 only).
-struct TcAttendArgs {
+struct alignas(64) TcAttendArgs {
+  CUtensorMap tmap_k;          // K as [b*g][N][d], 64x64 boxes, 128B swizzle (set by the launcher)
+  CUtensorMap tmap_v;          // V, likewise
   const __nv_bfloat16* q;      // [b,h,N,d]
   const __nv_bfloat16* k;      // [b,g,N,d]
   const __nv_bfloat16* v;
