@@ -411,17 +411,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       while (next_pv < n_items) {
         bool progressed = false;
         if (next_s < n_items && next_s < next_pv + NP &&
-            tc::mbar_test(tc::smem_u32(&bar_full_qk[next_s % NS]), (uint32_t)((next_s / NS) & 1))) {
+            tc::mbar_probe(tc::smem_u32(&bar_full_qk[next_s % NS]), (uint32_t)((next_s / NS) & 1))) {
           tc::fence_after_sync();
           issue_s(next_s);
           ++next_s;
           progressed = true;
         }
         if (next_pv < next_s &&
-            tc::mbar_test(tc::smem_u32(&bar_pfull[next_pv % NP]), (uint32_t)((next_pv / NP) & 1)) &&
-            tc::mbar_test(tc::smem_u32(&bar_full_v[next_pv % NS]), (uint32_t)((next_pv / NS) & 1)) &&
+            tc::mbar_probe(tc::smem_u32(&bar_pfull[next_pv % NP]), (uint32_t)((next_pv / NP) & 1)) &&
+            tc::mbar_probe(tc::smem_u32(&bar_full_v[next_pv % NS]), (uint32_t)((next_pv / NS) & 1)) &&
             (next_pv < 2 ||
-             tc::mbar_test(tc::smem_u32(&bar_ofree[next_pv & 1]), (uint32_t)(((next_pv - 2) >> 1) & 1)))) {
+             tc::mbar_probe(tc::smem_u32(&bar_ofree[next_pv & 1]), (uint32_t)(((next_pv - 2) >> 1) & 1)))) {
           tc::fence_after_sync();
           issue_pv(next_pv);
           ++next_pv;
@@ -608,41 +608,62 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       if (!wait(&bar_ofull[o], (uint32_t)((i >> 1) & 1))) break;
       if (!wait(&bar_mfull[i & 3], (uint32_t)((i >> 2) & 1))) break;
       tc::fence_after_sync();
-      if (wq * 32 < n_rows) {
-        const bool row_ok = t < n_rows;
-        int r = 0, slot;
-        float mult = 0.f;
-        if (row_ok) {
-          row_of(own, c, t0, t, r, slot);
-          mult = s_mult[i & 3][t];
-        }
+      const bool warp_ok = wq * 32 < n_rows;
+      const bool row_ok = t < n_rows;
+      int r = 0, slot;
+      float mult = 0.f;
+      if (row_ok) {
+        row_of(own, c, t0, t, r, slot);
+        mult = s_mult[i & 3][t];
+      }
+      // read-modify-write of 64 accumulator columns from a 64-column TMEM slice
+      auto accumulate = [&](const float* v, int c0) {
+        float4 u[8];
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tc::tmem_ld32(tO0 + o * D + c0 + lane_off, v);
-          tc::tmem_wait_ld();
-          if (row_ok) {
-            float4 u[8];
-            if (!own) {
+        for (int h = 0; h < 64; h += 32) {
+          if (!own) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) u[j] = *o_row_f4(sm, L.o, r, (c0 >> 2) + j, D);
-            } else {
+            for (int j = 0; j < 8; ++j) u[j] = *o_row_f4(sm, L.o, r, ((c0 + h) >> 2) + j, D);
+          } else {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) u[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            for (int j = 0; j < 8; ++j) u[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              u[j].x = fmaf(v[4 * j], mult, u[j].x);
-              u[j].y = fmaf(v[4 * j + 1], mult, u[j].y);
-              u[j].z = fmaf(v[4 * j + 2], mult, u[j].z);
-              u[j].w = fmaf(v[4 * j + 3], mult, u[j].w);
-              *o_row_f4(sm, L.o, r, (c0 >> 2) + j, D) = u[j];
-            }
+          for (int j = 0; j < 8; ++j) {
+            u[j].x = fmaf(v[h + 4 * j], mult, u[j].x);
+            u[j].y = fmaf(v[h + 4 * j + 1], mult, u[j].y);
+            u[j].z = fmaf(v[h + 4 * j + 2], mult, u[j].z);
+            u[j].w = fmaf(v[h + 4 * j + 3], mult, u[j].w);
+            *o_row_f4(sm, L.o, r, ((c0 + h) >> 2) + j, D) = u[j];
           }
         }
+      };
+      if constexpr (D == 64) {
+        // the whole tile row leaves TMEM at once, so the slot is released before the
+        // shared-memory read-modify-write
+        float v[64];
+        if (warp_ok) {
+          tc::tmem_ld32(tO0 + o * D + lane_off, v);
+          tc::tmem_ld32(tO0 + o * D + 32 + lane_off, v + 32);
+          tc::tmem_wait_ld();
+        }
+        tc::fence_before_sync();
+        mbar_arrive(tc::smem_u32(&bar_ofree[o]));
+        if (row_ok) accumulate(v, 0);
+      } else {
+        if (warp_ok) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 64) {
+            float v[64];
+            tc::tmem_ld32(tO0 + o * D + c0 + lane_off, v);
+            tc::tmem_ld32(tO0 + o * D + c0 + 32 + lane_off, v + 32);
+            tc::tmem_wait_ld();
+            if (row_ok) accumulate(v, c0);
+          }
+        }
+        tc::fence_before_sync();
+        mbar_arrive(tc::smem_u32(&bar_ofree[o]));
       }
-      tc::fence_before_sync();
-      mbar_arrive(tc::smem_u32(&bar_ofree[o]));
       // a row sits at different tile positions in different items: finish this item's
       // read-modify-writes before any epilogue warp starts the next one
       named_bar(2, 128);
