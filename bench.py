@@ -211,7 +211,7 @@ def run_prefill(args, ws_world, rank, local):
         st = ctypes.c_void_p(stream.cuda_stream)
         r = lib.hils_summarize(ctypes.byref(sh), P(k), P(lm), P(kb), P(hbb), st)
         if evs: evs[1].record(stream)
-        r |= lib.hils_select(ctypes.byref(sh), P(q), P(kb), P(hbb), P(idx), P(ssel), None, 0, st)
+        r |= lib.hils_select(ctypes.byref(sh), P(q), P(kb), P(hbb), P(idx), P(ssel), P(ws_sel), ws_sel.numel(), st)
         if evs: evs[2].record(stream)
         r |= lib.hils_attend_selected(ctypes.byref(sh), P(q), P(k), P(v), P(idx), P(ssel), P(out),
                                       P(ws_sel), ws_sel.numel(), st)

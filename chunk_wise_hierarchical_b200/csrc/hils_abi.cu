@@ -128,7 +128,7 @@ hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) 
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   switch (op) {
-    case HILS_OP_SELECT: *bytes = 0; return HILS_OK;
+    case HILS_OP_SELECT: *bytes = kHeader; return HILS_OK;
     case HILS_OP_ATTEND: *bytes = attend_layout(s).total; return HILS_OK;
     case HILS_OP_DECODE: *bytes = decode_layout(s).total; return HILS_OK;
     case HILS_OP_ATTEND_SELECTED: *bytes = kHeader; return HILS_OK;
@@ -169,20 +169,27 @@ hils_status hils_summarize_paged(const hils_shape* s, const void* k_pages, const
   return cuda_status(hils::run_summarize(a, (cudaStream_t)stream));
 }
 
+// Scores + Top-K: the tensor-core kernel where it applies (bf16, G = 1), else SIMT.
+static cudaError_t run_select(const hils::SelectArgs& a, cudaStream_t st) {
+  if (hils::select_tc_supported(a.d, a.h / a.g, a.top_k, a.bf16)) return hils::run_select_tc(a, st);
+  return hils::run_select_simt(a, st);
+}
+
 hils_status hils_select(const hils_shape* s, const void* q, const float* kbar, const float* hbias,
                         int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws; (void)ws_bytes;
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if ((size_t)s->batch * s->seq_len * s->top_k == 0) return HILS_OK;
   const int C = s->seq_len / s->chunk;
   if (!q || !topk_idx || (C > 0 && (!kbar || !hbias))) return HILS_ERR_INVALID_ARG;
-  if (!aligned16(q)) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || (C > 0 && !aligned16(kbar))) return HILS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
   hils::SelectArgs a{};
   a.q = q; a.kbar = kbar; a.hbias = hbias; a.idx = topk_idx; a.score = topk_score;
+  a.err = static_cast<unsigned*>(ws);
   a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
   a.n_chunks = C; a.top_k = s->top_k; a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
-  return cuda_status(hils::run_select_simt(a, (cudaStream_t)stream));
+  return cuda_status(run_select(a, (cudaStream_t)stream));
 }
 
 hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const void* v,
@@ -219,7 +226,8 @@ hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const
     se.q = q; se.kbar = kbar; se.hbias = hbias; se.idx = idx; se.score = ssel;
     se.b = s->batch; se.h = s->heads_q; se.g = s->heads_kv; se.n = s->seq_len; se.d = s->head_dim;
     se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16;
-    if (hils::run_select_simt(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
+    se.err = reinterpret_cast<unsigned*>(w);
+    if (run_select(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
   }
   return cuda_status(run_prefill_attention(s, q, k, v, idx, ssel, out, reinterpret_cast<unsigned*>(w), cs));
 }

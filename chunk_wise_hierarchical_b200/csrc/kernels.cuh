@@ -28,11 +28,15 @@ struct SelectArgs {
   const float* hbias;     // [b,h,C]
   int32_t* idx;           // [b,g,N,K]
   float* score;           // [b,h,N,K] or nullptr
+  unsigned* err;          // sticky error word or nullptr
   int b, h, g, n, d, n_chunks, top_k;
   float scale;
   bool bf16;
 };
 cudaError_t run_select_simt(const SelectArgs& a, cudaStream_t st);
+// Tensor-core scores + Top-K (bf16, one query head per KV head).
+bool select_tc_supported(int d, int G, int K, bool bf16);
+cudaError_t run_select_tc(const SelectArgs& a, cudaStream_t st);
 
 // Paged decode: split scan + Top-K (last CTA merges), then per-chunk attention
 // with a last-CTA fusion, chained by programmatic dependent launch.

@@ -143,8 +143,12 @@ HILS_API hils_status hils_summarize_paged(const hils_shape* shape, const void* k
  *               descending key order; slots >= K_eff hold -1
  *   topk_score  [batch, heads_q, seq_len, top_k] fp32 or NULL: each head's
  *               own shat of the selected chunks (-inf in unused slots)
- *   ws          workspace of hils_workspace_size(HILS_OP_SELECT) bytes
- *               (may be NULL when that size is 0)
+ *   ws          workspace of hils_workspace_size(HILS_OP_SELECT) bytes,
+ *               zero-filled before first use: it holds only the sticky
+ *               error word read by hils_device_status
+ * kbar must be 16-byte aligned.  For bf16 with heads_q == heads_kv the
+ * scores run on the tensor cores with the fp32 summaries split into two
+ * bf16 parts (score error near 2^-17 |q||kbar|).
  */
 HILS_API hils_status hils_select(const hils_shape* shape, const void* q, const float* kbar,
                         const float* hbias, int32_t* topk_idx, float* topk_score, void* ws,

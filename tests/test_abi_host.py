@@ -48,7 +48,7 @@ def test_workspace_sizes():
     C = 1000 // 64
     need = 2 * 8 * C * 64 * 4 + 2 * 8 * C * 4 + 2 * 2 * 1000 * 16 * 4 + 2 * 8 * 1000 * 16 * 4
     assert need <= n <= need + 6 * 256
-    assert _abi.workspace_size(s, _abi.OP_SELECT) == 0
+    assert _abi.workspace_size(s, _abi.OP_SELECT) == 256
     assert _abi.workspace_size(s, _abi.OP_DECODE) >= 2 * 2 * 16 * 8
 
 
@@ -75,6 +75,7 @@ def test_entry_points_reject_before_launch():
     assert lib.hils_attend(ctypes.byref(s), P((1 << 20) + 4), fake, fake, fake, fake, None, fake,
                            1 << 30, None) == 1  # misaligned
     assert lib.hils_select(ctypes.byref(s), fake, None, fake, fake, None, None, 0, None) == 1
+    assert lib.hils_select(ctypes.byref(s), fake, fake, fake, fake, None, None, 0, None) == 3  # no error word
     assert lib.hils_summarize(ctypes.byref(s), fake, None, fake, fake, None) == 1
     assert lib.hils_summarize_paged(ctypes.byref(s), fake, fake, fake, -1, 4, fake, fake, None) == 1
     assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 0, fake, 4, fake, None,

@@ -91,6 +91,33 @@ def test_summaries_and_select_match_oracle():
                     assert abs(gsc[0, h, i, s] - shat[0, h, i, c]) < 1e-4
 
 
+@pytest.mark.parametrize("kw", [
+    dict(batch=1, heads_q=2, heads_kv=2, seq_len=64 * 260 + 17, head_dim=64, top_k=16, needles=8),
+    dict(batch=2, heads_q=1, heads_kv=1, seq_len=64 * 140 + 5, head_dim=128, top_k=64, qkv_std=0.5),
+    dict(batch=1, heads_q=1, heads_kv=1, seq_len=64 * 129, head_dim=64, top_k=1),
+])
+def test_select_one_head_per_group_bf16(kw):
+    """bf16 with G = 1 scores on the tensor cores (split-bf16 summaries):
+    indices as the oracle's up to near-ties, scores within 1e-4."""
+    inp = prefill_inputs(dtype="bf16", seed=21, **kw)
+    K, g = kw["top_k"], kw["heads_kv"]
+    kbar, hb = hils.summarize(inp.k.cuda(), inp.landmark.cuda())
+    rk, rh = O.summarize(inp.k, inp.landmark, 64)
+    idx, sc = hils.select(inp.q.cuda(), kbar, hb, K, g)
+    shat = O.chunk_scores(inp.q, rk, rh, 64)
+    _, key = O.select_topk(shat, g, K)
+    gi = idx.cpu().numpy()
+    check_indices(gi, key, K)
+    gsc = sc.cpu().numpy()
+    b_, h_, n_, _ = gsc.shape
+    bi, hi, ii, si = np.nonzero(gi >= 0)
+    want = shat[bi, hi, ii, gi[bi, hi, ii, si]]
+    assert np.abs(gsc[bi, hi, ii, si] - want).max() < 1e-4
+    assert np.all(gsc[gi < 0] == -np.inf)
+    n_eff = np.minimum(np.arange(n_) // 64, K)
+    assert np.array_equal((gi >= 0).sum(-1), np.broadcast_to(n_eff, (b_, h_, n_)))
+
+
 def _rows_sample(n, rng, count=40):
     edge = [0, 1, 63, 64, 65, 127, 128, n // 2, n - 65, n - 64, n - 2, n - 1]
     return np.unique(np.concatenate([edge, rng.integers(0, n, count)]))
