@@ -16,6 +16,7 @@ from ._abi import (  # noqa: F401
     OP_DECODE,
     OP_ATTEND_SELECTED,
     decode,
+    decode_static,
     select,
     summarize,
     summarize_paged,

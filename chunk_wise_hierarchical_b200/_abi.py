@@ -65,6 +65,7 @@ def lib():
         "hils_attend": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "hils_attend_selected": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "hils_decode": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
+        "hils_decode_static": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, _P]),
         "hils_device_status": (i32, [_P, _P]),
     }
     for name, (res, args) in sig.items():
@@ -76,7 +77,7 @@ def lib():
 
 
 EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_decode",
-            "hils_device_status", "hils_select", "hils_status_string", "hils_summarize",
+            "hils_decode_static", "hils_device_status", "hils_select", "hils_status_string", "hils_summarize",
             "hils_summarize_paged", "hils_workspace_size"]
 
 
@@ -257,3 +258,27 @@ def decode(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, 
     out = call(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, topk_idx=idx,
                stream=stream)
     return (out, idx) if return_idx else out
+
+
+DECODE_STATIC_SCRATCH_BYTES = 4 << 20
+
+
+def decode_static(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, top_k,
+                  scale=None, out=None, topk_idx=None, status_word=None, stream=None):
+    """hils_decode_static: decode without a workspace (the library's own
+    scratch array is used).  Calls on one device must not overlap in time."""
+    b, h, d = q.shape
+    g = k_pages.shape[1]
+    max_chunks = block_table.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_table and seq_lens must be int32")
+    if status_word is not None and (status_word.dtype != torch.int32 or status_word.numel() < 1):
+        raise TypeError("status_word must be an int32 device tensor")
+    sh = make_shape(b, h, g, d, max_chunks * 64, top_k, _dt(q), scale=scale or 0.0)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().hils_decode_static(ctypes.byref(sh), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kbar_pages),
+                                    _ptr(hbias_pages), _ptr(block_table), max_chunks, _ptr(seq_lens),
+                                    int(k_pages.shape[0]), _ptr(out), _ptr(topk_idx), _ptr(status_word),
+                                    _stream(stream)), "hils_decode_static")
+    return out

@@ -4,6 +4,7 @@
 // (except hils_device_status).
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/hils.h"
 #include "common.cuh"
@@ -296,6 +297,111 @@ hils_status hils_device_status(void* ws, void* stream) {
   if (word & hils::kErrTimeout) return HILS_ERR_DEVICE_TIMEOUT;
   if (word & hils::kErrBadPage) return HILS_ERR_DEVICE_CHECK;
   return HILS_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// hils_decode_static: decode whose scratch is a device array owned by this
+// file, for callers that cannot hand the library a workspace (no counterpart
+// in the HiLS notes).  Nothing here allocates or frees device memory.
+namespace {
+
+constexpr size_t kStaticScratchBytes = HILS_DECODE_STATIC_SCRATCH_BYTES;
+constexpr size_t kStaticTicketSlots = 4096;  // batch * heads_kv limit
+constexpr int kStaticMaxDevices = 64;
+
+// Scratch of hils_decode_static.  Byte layout (fixed parts first, so the ticket
+// counters never share bytes with the data of a call of another shape):
+//   [0, 256)                 error word, when the caller passes no status word
+//   [256, 256 + 16 KiB)      scan tickets, one per (sequence, KV head)
+//   [.., + 16 KiB)           attention tickets
+//   then, per call's shape: part_keys, part_att, idx, sel_page, ssel
+// The ticket counters must be zero when a call starts: device memory of a
+// __device__ array is zero when the module is loaded, and every call that
+// completes leaves them at zero (the CTA that consumes a ticket resets it).
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+struct StaticLayout {
+  size_t scan_ticket, att_ticket, part_keys, part_att, idx, sel_page, ssel, total;
+};
+StaticLayout static_decode_layout(const hils_shape* s) {
+  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k, d = s->head_dim;
+  const size_t G = h / g;
+  const int cmax = (s->seq_len + s->chunk - 1) / s->chunk;
+  const size_t nsplit = hils::decode_splits(cmax);
+  StaticLayout L;
+  size_t off = kHeader;
+  L.scan_ticket = off; off += kStaticTicketSlots * 4;
+  L.att_ticket = off; off += kStaticTicketSlots * 4;
+  L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
+  L.part_att = off; off = align_up(off + b * g * (K + 1) * G * (d + 2) * 4);
+  L.idx = off; off = align_up(off + b * g * K * 4);
+  L.sel_page = off; off = align_up(off + b * g * K * 4);
+  L.ssel = off; off = align_up(off + b * h * K * 4);
+  L.total = off;
+  return L;
+}
+
+std::mutex g_static_mu;
+unsigned char* g_static_ptr[kStaticMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the lookup may load this library's device code onto it).
+cudaError_t static_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kStaticMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k_pages, const void* v_pages,
+                               const float* kbar_pages, const float* hbias_pages, const int32_t* block_table,
+                               int32_t max_chunks, const int32_t* seq_lens, int32_t n_pages, void* out,
+                               int32_t* topk_idx_out, unsigned* status_word, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if (s->batch == 0) return HILS_OK;
+  if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
+  if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
+  if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
+    return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(kbar_pages) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(status_word) & 3u) != 0)
+    return HILS_ERR_INVALID_ARG;
+  if ((size_t)s->batch * s->heads_kv > kStaticTicketSlots) return HILS_ERR_WORKSPACE;
+  const StaticLayout L = static_decode_layout(s);
+  if (L.total > kStaticScratchBytes) return HILS_ERR_WORKSPACE;
+  unsigned char* w = nullptr;
+  if (static_scratch(&w) != cudaSuccess) return HILS_ERR_CUDA;
+  hils::DecodeArgs da{};
+  da.q = q; da.k_pages = k_pages; da.v_pages = v_pages; da.kbar_pages = kbar_pages;
+  da.hbias_pages = hbias_pages; da.block_table = block_table; da.seq_lens = seq_lens; da.out = out;
+  da.idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(w + L.idx);
+  da.ssel = reinterpret_cast<float*>(w + L.ssel);
+  da.sel_page = reinterpret_cast<int32_t*>(w + L.sel_page);
+  da.part_keys = reinterpret_cast<unsigned long long*>(w + L.part_keys);
+  da.part_att = reinterpret_cast<float*>(w + L.part_att);
+  da.scan_ticket = reinterpret_cast<unsigned*>(w + L.scan_ticket);
+  da.att_ticket = reinterpret_cast<unsigned*>(w + L.att_ticket);
+  da.err = status_word ? status_word : reinterpret_cast<unsigned*>(w);
+  da.b = s->batch; da.h = s->heads_q; da.g = s->heads_kv; da.d = s->head_dim; da.top_k = s->top_k;
+  da.max_chunks = max_chunks; da.n_pages = n_pages; da.scale = eff_scale(s);
+  da.bf16 = s->dtype == HILS_BF16;
+  return cuda_status(hils::run_decode(da, (cudaStream_t)stream));
 }
 
 }  // extern "C"

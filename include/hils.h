@@ -217,6 +217,41 @@ HILS_API hils_status hils_decode(const hils_shape* shape, const void* q, const v
                         size_t ws_bytes, void* stream);
 
 /*
+ * hils_decode_static -- hils_decode with no workspace argument.  The HiLS
+ * notes have no counterpart: this is a plumbing variant for callers that
+ * cannot hand the library a device buffer, e.g. an engine whose device memory
+ * is carved up once at start-up, or a loop that must not call cudaMalloc or
+ * cudaFree, which can synchronise the whole device and stall its other
+ * streams.  The call itself allocates and frees nothing: its scratch is one
+ * fixed device array of HILS_DECODE_STATIC_SCRATCH_BYTES bytes inside
+ * libhils.so.
+ *   Arguments as for hils_decode, except:
+ *   status_word  NULL, or a 4-byte-aligned device word, zero-filled by the
+ *                caller, into which the kernels OR their error bits (read
+ *                and clear it with hils_device_status(status_word, stream));
+ *                with NULL, device-side errors are not reported
+ * Returns HILS_ERR_WORKSPACE, without launching anything, when the shape
+ * needs more scratch than the array holds (batch * heads_kv > 4096, or
+ * roughly 256 + 32 KiB + what hils_workspace_size(HILS_OP_DECODE) reports
+ * beyond its own 256-byte header > HILS_DECODE_STATIC_SCRATCH_BYTES).
+ * The first call on each device looks up the array's device address (this
+ * may load the library's device code onto that device): make it before any
+ * stream capture starts.
+ * Every call on a device uses the same array: calls whose kernels may run at
+ * the same time (different streams with no ordering between them, or
+ * different host threads) race on it and corrupt each other's results; order
+ * them on one stream or with events.  Its ticket counters must start at zero:
+ * they are zero when the library's device code is loaded, and each call that
+ * completes leaves them at zero again.
+ */
+#define HILS_DECODE_STATIC_SCRATCH_BYTES (4u << 20)
+HILS_API hils_status hils_decode_static(const hils_shape* shape, const void* q, const void* k_pages,
+                        const void* v_pages, const float* kbar_pages, const float* hbias_pages,
+                        const int32_t* block_table, int32_t max_chunks, const int32_t* seq_lens,
+                        int32_t n_pages, void* out, int32_t* topk_idx_out, unsigned* status_word,
+                        void* stream);
+
+/*
  * hils_device_status -- synchronises `stream`, reads and clears the error
  * word at the start of a hils_attend / hils_attend_selected / hils_decode
  * workspace, and returns HILS_OK, HILS_ERR_DEVICE_CHECK or
