@@ -120,22 +120,28 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(args=None, backend="nccl"):
+    """One process per GPU under torchrun; returns (world size, rank, local rank)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=300)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=timeout)
     return ws, rank, local
 
 
 def max_over_ranks(x, ws):
+    """Max of a per-rank time over all ranks (every rank gets the result)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -143,7 +149,13 @@ def max_over_ranks(x, ws):
 def barrier(ws):
     if ws > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def job_tflops(ws, flops_per_replica, ms_max):
+    """Whole-job throughput of ws replicas that each do flops_per_replica in (max) ms_max."""
+    return ws * flops_per_replica / (ms_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------------------- CPU baseline (oracle)
@@ -338,7 +350,7 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
         return
     flops = pre["flops"]
-    value = ws_world * flops / (pre["ms_step"] * 1e-3) / 1e12
+    value = job_tflops(ws_world, flops, pre["ms_step"])
     att_tflops = flops / (pre["ms_att"] * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -364,7 +376,7 @@ def run_ours(args):
                      "achieved": round(att_tflops, 3), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": round(att_tflops / bf16_peak, 5), "peak_source": f"{peak_src} bf16 burst",
                      "traffic": args.traffic},
-        "e2e": {"value": round(ws_world * flops / (pre["ms_e2e"] * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+        "e2e": {"value": round(job_tflops(ws_world, flops, pre["ms_e2e"]), 4), "unit": "TFLOP/s",
                 "ms_per_step": round(pre["ms_e2e"], 3), "h2d_bytes_per_step": pre["h2d"],
                 "d2h_bytes_per_step": pre["d2h"]},
         "gpu_launches": pre["launches_per_step"] * args.steps,
