@@ -61,7 +61,7 @@ struct TcCfg {
 };
 
 struct TcSmem {
-  uint32_t stage, p, o, list, off, items, rowm, rowz, total;
+  uint32_t stage, o, list, off, items, rowm, rowz, total;
 };
 
 __host__ __device__ inline uint32_t align_to(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -77,7 +77,6 @@ __host__ __device__ inline TcSmem tc_layout(int G, int qb, int K, int n_cand) {
   TcSmem L;
   uint32_t off = 0;
   L.stage = off; off += C::NS * C::kStageStride;
-  L.p = off; off += C::NP * 128 * 64 * 2;
   L.o = off; off += (uint32_t)qb * G * D * 4;
   L.list = off; off = align_to(off + (uint32_t)qb * K * 2, 16);
   L.off = off; off = align_to(off + (uint32_t)(2 * n_cand + 2) * 4, 16);
@@ -394,13 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       };
       auto issue_pv = [&](int i) {
         const int s = i % NS, b = i % NP, o = i & 1;
-        const uint32_t sP = tc::smem_u32(sm + L.p + b * 16384);
         const uint32_t sV = tc::smem_u32(stage_ptr(s)) + C::kStageA + C::kStageK;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t da = tc::make_desc(sP + k * 32u, 16, 1024);
+          // P (bf16) sits in the first 32 columns of S's slot: 16 keys = 8 columns per step
           const uint64_t db = tc::make_desc(sV + k * 2048u, 8192, 1024);
-          tc::mma_bf16(tO0 + o * D, da, db, idO, k > 0);
+          tc::mma_bf16_tmem_a(tO0 + o * D, tS0 + b * 64 + k * 8, db, idO, k > 0);
         }
         tc::mma_commit(tc::smem_u32(&bar_ofull[o]));
       };
@@ -490,7 +488,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     bool synced_own = false;
     for (int i = wg; i < n_items && wg < NP; i += NP) {
       const int b = i % NP;
-      bool ok_loop = true;
       int c, t0, n_rows;
       bool own;
       item_rows(s_items[i], c, own, t0, n_rows);
@@ -566,32 +563,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             mult = expf(sh - s_rowm[r]) * s_rowz[r] / l;
           }
         }
-        // P slot b was last read by P.V(i - NP): it must have completed before it is
-        // overwritten (S(i) completing does not imply it)
-        if (i >= NP && !wait(&bar_ofull[(i - NP) & 1], (uint32_t)(((i - NP) >> 1) & 1))) {
-          ok_loop = false;
-        }
-        if (row_ok && ok_loop) {
-          s_mult[i & 3][t] = mult;
-          unsigned char* prow = sm + L.p + b * 16384;
+        // P overwrites the first 32 columns of S's slot (this lane's row, already in
+        // registers).  P.V(i - NP), the last reader of the slot, was issued before S(i)
+        // and tcgen05 MMAs run in issue order, so the slot is free.
+        if (row_ok) s_mult[i & 3][t] = mult;
+        uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 64; j += 8) {
-            uint4 pk;
-            pk.x = tc::pack_bf16x2(s[j], s[j + 1]);
-            pk.y = tc::pack_bf16x2(s[j + 2], s[j + 3]);
-            pk.z = tc::pack_bf16x2(s[j + 4], s[j + 5]);
-            pk.w = tc::pack_bf16x2(s[j + 6], s[j + 7]);
-            *reinterpret_cast<uint4*>(prow + tc::sw128_chunk(t, j >> 3)) = pk;
-          }
-        }
+        for (int j = 0; j < 32; ++j) pk[j] = tc::pack_bf16x2(s[2 * j], s[2 * j + 1]);
+        tc::tmem_st32(tmem + b * 64 + lane_off, pk);
+        tc::tmem_wait_st();
       }
-      tc::fence_async_smem();
       tc::fence_before_sync();
       mbar_arrive(tc::smem_u32(&bar_pfull[b]));
       // the epilogue of item i reads s_mult[i & 3]; it cannot lap this ring: item i + 4
       // needs S(i+4), which waits for P.V(i+2), which waits for that epilogue
       mbar_arrive(tc::smem_u32(&bar_mfull[i & 3]));
-      if (!ok_loop) break;
     }
     if (!synced_own) named_bar(1, 256);
   } else if (warp >= 12) {
