@@ -95,6 +95,19 @@ __device__ __forceinline__ float4* o_row_f4(unsigned char* base, uint32_t o_off,
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Named barrier that also returns the OR of `pred` over the participating threads.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -147,12 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   static_assert(NS == NP, "stage and S-slot rings must have the same depth");
   __shared__ uint64_t bar_full_qk[NS], bar_full_v[NS];
   __shared__ uint64_t bar_sfull[NP], bar_pfull[NP], bar_ofull[2], bar_ofree[2];
-  __shared__ uint64_t bar_mfull[4];  // the item's row multipliers are written (ring of 4 items)
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_wsum[kThreads / 32];
   __shared__ int s_n_items;
   __shared__ volatile int s_abort;
-  __shared__ float s_mult[4][128];  // per item (ring of 4) and tile row: epilogue multiplier
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = a.n, K = a.top_k, QB = a.qb;
@@ -192,7 +203,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       tc::mbar_init(tc::smem_u32(&bar_ofull[s]), 1);
       tc::mbar_init(tc::smem_u32(&bar_ofree[s]), 128);
     }
-    for (int s = 0; s < 4; ++s) tc::mbar_init(tc::smem_u32(&bar_mfull[s]), 128);
     tc::mbar_fence_init();
     s_abort = 0;
   }
@@ -507,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         tc::tmem_ld32(tmem + b * 64 + lane_off, s);
         tc::tmem_ld32(tmem + b * 64 + 32 + lane_off, s + 32);
         tc::tmem_wait_ld();
-        float mult;  // applied by the epilogue: O_tile row * mult
+        float mult;  // the row's fusion factor, folded into P so that P.V is the final term
         if (!own && sc2 > 0.f) {
           // lean path (all 64 keys valid): raw max, p = exp2(S*c - m*c), one FFMA + ex2 each
           float mp[8];
@@ -563,21 +573,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
             mult = expf(sh - s_rowm[r]) * s_rowz[r] / l;
           }
         }
-        // P overwrites the first 32 columns of S's slot (this lane's row, already in
-        // registers).  P.V(i - NP), the last reader of the slot, was issued before S(i)
+        // P = mult * p overwrites the first 32 columns of S's slot (this lane's row, already
+        // in registers).  P.V(i - NP), the last reader of the slot, was issued before S(i)
         // and tcgen05 MMAs run in issue order, so the slot is free.
-        if (row_ok) s_mult[i & 3][t] = mult;
         uint32_t pk[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = tc::pack_bf16x2(s[2 * j], s[2 * j + 1]);
+        for (int j = 0; j < 32; ++j) pk[j] = tc::pack_bf16x2(s[2 * j] * mult, s[2 * j + 1] * mult);
         tc::tmem_st32(tmem + b * 64 + lane_off, pk);
         tc::tmem_wait_st();
       }
       tc::fence_before_sync();
       mbar_arrive(tc::smem_u32(&bar_pfull[b]));
-      // the epilogue of item i reads s_mult[i & 3]; it cannot lap this ring: item i + 4
-      // needs S(i+4), which waits for P.V(i+2), which waits for that epilogue
-      mbar_arrive(tc::smem_u32(&bar_mfull[i & 3]));
     }
     if (!synced_own) named_bar(1, 256);
   } else if (warp >= 12) {
@@ -586,73 +592,90 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     const int wq = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     const uint32_t tO0 = tmem + NP * 64;
-    for (int i = 0; i < n_items; ++i) {
-      const int o = i & 1;
-      int c, t0, n_rows;
-      bool own;
-      item_rows(s_items[i], c, own, t0, n_rows);
-      if (!wait(&bar_ofull[o], (uint32_t)((i >> 1) & 1))) break;
-      if (!wait(&bar_mfull[i & 3], (uint32_t)((i >> 2) & 1))) break;
-      tc::fence_after_sync();
-      const bool warp_ok = wq * 32 < n_rows;
-      const bool row_ok = t < n_rows;
-      int r = 0, slot;
-      float mult = 0.f;
-      if (row_ok) {
-        row_of(own, c, t0, t, r, slot);
-        mult = s_mult[i & 3][t];
+    struct Geo {
+      bool own, warp_ok, row_ok;
+      int r;
+    };
+    auto geo = [&](int i) {
+      int c, t0, n_rows, slot;
+      Geo g;
+      item_rows(s_items[i], c, g.own, t0, n_rows);
+      g.warp_ok = wq * 32 < n_rows;
+      g.row_ok = t < n_rows;
+      g.r = 0;
+      if (g.row_ok) row_of(g.own, c, t0, t, g.r, slot);
+      return g;
+    };
+    // acc[r] (own item: =, selected chunk: +=) the tile row's columns [c0, c0 + 32) in v;
+    // P already carries the fusion factor, so the tile row is the final term
+    auto add32 = [&](const float* v, const Geo& g, int c0) {
+      float4 u[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        u[j] = g.own ? make_float4(0.f, 0.f, 0.f, 0.f) : *o_row_f4(sm, L.o, g.r, (c0 >> 2) + j, D);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        u[j].x += v[4 * j];
+        u[j].y += v[4 * j + 1];
+        u[j].z += v[4 * j + 2];
+        u[j].w += v[4 * j + 3];
+        *o_row_f4(sm, L.o, g.r, (c0 >> 2) + j, D) = u[j];
       }
-      // read-modify-write of 64 accumulator columns from a 64-column TMEM slice
-      auto accumulate = [&](const float* v, int c0) {
-        float4 u[8];
-#pragma unroll
-        for (int h = 0; h < 64; h += 32) {
-          if (!own) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) u[j] = *o_row_f4(sm, L.o, r, ((c0 + h) >> 2) + j, D);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) u[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            u[j].x = fmaf(v[h + 4 * j], mult, u[j].x);
-            u[j].y = fmaf(v[h + 4 * j + 1], mult, u[j].y);
-            u[j].z = fmaf(v[h + 4 * j + 2], mult, u[j].z);
-            u[j].w = fmaf(v[h + 4 * j + 3], mult, u[j].w);
-            *o_row_f4(sm, L.o, r, ((c0 + h) >> 2) + j, D) = u[j];
-          }
-        }
-      };
-      if constexpr (D == 64) {
-        // the whole tile row leaves TMEM at once, so the slot is released before the
-        // shared-memory read-modify-write
-        float v[64];
-        if (warp_ok) {
-          tc::tmem_ld32(tO0 + o * D + lane_off, v);
-          tc::tmem_ld32(tO0 + o * D + 32 + lane_off, v + 32);
-          tc::tmem_wait_ld();
-        }
+    };
+    // A row sits at different tile positions in different items, so every item's
+    // read-modify-writes finish (named barrier 2) before the next item's start.  The
+    // barrier also votes on leaving the loop, so all 128 threads leave together.
+    if constexpr (D == 64) {
+      // 32-column halves in a software pipeline: the TMEM load of the next half runs
+      // while the previous half is added into shared memory
+      float va[32], vb[32];
+      bool ok = true;
+      Geo cur{};
+      if (n_items > 0) {
+        ok = __all_sync(0xffffffffu, wait(&bar_ofull[0], 0u));
+        tc::fence_after_sync();
+        cur = geo(0);
+        if (ok && cur.warp_ok) tc::tmem_ld32(tO0 + lane_off, va);
+        tc::tmem_wait_ld();
+      }
+      for (int i = 0; i < n_items; ++i) {
+        const int o = i & 1;
+        if (ok && cur.warp_ok) tc::tmem_ld32(tO0 + o * 64 + 32 + lane_off, vb);
+        if (ok && cur.row_ok) add32(va, cur, 0);
+        tc::tmem_wait_ld();
         tc::fence_before_sync();
-        mbar_arrive(tc::smem_u32(&bar_ofree[o]));
-        if (row_ok) accumulate(v, 0);
-      } else {
-        if (warp_ok) {
+        mbar_arrive(tc::smem_u32(&bar_ofree[o]));  // item i has left TMEM
+        Geo nxt{};
+        if (i + 1 < n_items) {
+          ok = __all_sync(0xffffffffu, ok && wait(&bar_ofull[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1)));
+          tc::fence_after_sync();
+          nxt = geo(i + 1);
+          if (ok && nxt.warp_ok) tc::tmem_ld32(tO0 + ((i + 1) & 1) * 64 + lane_off, va);
+        }
+        if (ok && cur.row_ok) add32(vb, cur, 32);
+        tc::tmem_wait_ld();
+        if (named_bar_or(2, 128, !ok || s_abort)) break;
+        cur = nxt;
+      }
+    } else {
+      for (int i = 0; i < n_items; ++i) {
+        const int o = i & 1;
+        const bool ok = __all_sync(0xffffffffu, wait(&bar_ofull[o], (uint32_t)((i >> 1) & 1)));
+        tc::fence_after_sync();
+        const Geo g = geo(i);
+        if (ok && g.warp_ok) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 64) {
-            float v[64];
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float v[32];
             tc::tmem_ld32(tO0 + o * D + c0 + lane_off, v);
-            tc::tmem_ld32(tO0 + o * D + c0 + 32 + lane_off, v + 32);
             tc::tmem_wait_ld();
-            if (row_ok) accumulate(v, c0);
+            if (g.row_ok) add32(v, g, c0);
           }
         }
         tc::fence_before_sync();
         mbar_arrive(tc::smem_u32(&bar_ofree[o]));
+        if (named_bar_or(2, 128, !ok || s_abort)) break;
       }
-      // a row sits at different tile positions in different items: finish this item's
-      // read-modify-writes before any epilogue warp starts the next one
-      named_bar(2, 128);
     }
   }
 
