@@ -51,10 +51,11 @@ constexpr uint32_t kOwnFlag = 0x80000000u;
 
 template <int D>
 struct TcCfg {
-  static constexpr int NS = D == 64 ? 2 : 1;         // operand stages
-  static constexpr int NP = D == 64 ? 2 : 1;         // S (TMEM) / P (smem) slots
+  static constexpr int NS = D == 64 ? 3 : 1;         // operand stages
+  static constexpr int NP = D == 64 ? 3 : 1;         // S / P slots (TMEM)
+  static constexpr int NO = D == 64 ? 3 : 2;         // P.V output slots (TMEM), >= NS
   static constexpr int kRows = D == 64 ? 384 : 256;  // target rows (QB * G) per CTA
-  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 512;  // NP S/P slots of 64 + NO output slots of D
   static constexpr uint32_t kStageA = 128 * D * 2, kStageK = 64 * D * 2, kStageV = 64 * D * 2;
   static constexpr uint32_t kStage = kStageA + kStageK + kStageV;
   static constexpr uint32_t kStageStride = (kStage + 1023) / 1024 * 1024;
@@ -150,7 +151,7 @@ __device__ int block_exclusive_scan(int* v, int n, int* wsum) {
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ TcAttendArgs a) {
   using C = TcCfg<D>;
-  constexpr int NS = C::NS, NP = C::NP;
+  constexpr int NS = C::NS, NP = C::NP, NO = C::NO;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                        ~static_cast<uintptr_t>(1023));
@@ -158,8 +159,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   // free once S of its item completed (sfull), its V half once P.V completed (ofull):
   // each MMA group is committed to exactly one barrier, which every consumer waits on
   static_assert(NS == NP, "stage and S-slot rings must have the same depth");
+  // the V producer waits for P.V(i - NS) on the output ring: with NO >= NS the barrier
+  // cannot run a full lap ahead of that wait (P.V(i - NS + NO) needs V(i))
+  static_assert(NO >= NS && C::NP * 64 + NO * D <= (int)C::kTmemCols, "output ring");
   __shared__ uint64_t bar_full_qk[NS], bar_full_v[NS];
-  __shared__ uint64_t bar_sfull[NP], bar_pfull[NP], bar_ofull[2], bar_ofree[2];
+  __shared__ uint64_t bar_sfull[NP], bar_pfull[NP], bar_ofull[NO], bar_ofree[NO];
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_wsum[kThreads / 32];
   __shared__ int s_n_items;
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       tc::mbar_init(tc::smem_u32(&bar_sfull[s]), 1);
       tc::mbar_init(tc::smem_u32(&bar_pfull[s]), 128);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NO; ++s) {
       tc::mbar_init(tc::smem_u32(&bar_ofull[s]), 1);
       tc::mbar_init(tc::smem_u32(&bar_ofree[s]), 128);
     }
@@ -374,8 +378,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     if (lane == 0) {
       for (int i = 0; i < n_items; ++i) {
         const int s = i % NS;
-        // P.V of item i - NS must have completed
-        if (i >= NS && !wait(&bar_ofull[(i - NS) & 1], (uint32_t)(((i - NS) >> 1) & 1))) break;
+        // P.V of item i - NS, the last reader of this stage's V, must have completed
+        if (i >= NS && !wait(&bar_ofull[(i - NS) % NO], (uint32_t)(((i - NS) / NO) & 1))) break;
         const int c = (int)((s_items[i] >> 16) & 0x7fffu);
         const uint32_t sV = tc::smem_u32(stage_ptr(s)) + C::kStageA + C::kStageK;
         const uint32_t full = tc::smem_u32(&bar_full_v[s]);
@@ -402,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         tc::mma_commit(tc::smem_u32(&bar_sfull[b]));
       };
       auto issue_pv = [&](int i) {
-        const int s = i % NS, b = i % NP, o = i & 1;
+        const int s = i % NS, b = i % NP, o = i % NO;
         const uint32_t sV = tc::smem_u32(stage_ptr(s)) + C::kStageA + C::kStageK;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -410,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
           const uint64_t db = tc::make_desc(sV + k * 2048u, 8192, 1024);
           tc::mma_bf16_tmem_a(tO0 + o * D, tS0 + b * 64 + k * 8, db, idO, k > 0);
         }
+        // one commit per MMA group: a second commit would track no MMA and arrive at once
         tc::mma_commit(tc::smem_u32(&bar_ofull[o]));
       };
       // event loop: issue S(next_s) as soon as its operands have landed and its S slot
@@ -428,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         if (next_pv < next_s &&
             tc::mbar_probe(tc::smem_u32(&bar_pfull[next_pv % NP]), (uint32_t)((next_pv / NP) & 1)) &&
             tc::mbar_probe(tc::smem_u32(&bar_full_v[next_pv % NS]), (uint32_t)((next_pv / NS) & 1)) &&
-            (next_pv < 2 ||
-             tc::mbar_probe(tc::smem_u32(&bar_ofree[next_pv & 1]), (uint32_t)(((next_pv - 2) >> 1) & 1)))) {
+            (next_pv < NO ||
+             tc::mbar_probe(tc::smem_u32(&bar_ofree[next_pv % NO]), (uint32_t)(((next_pv - NO) / NO) & 1)))) {
           tc::fence_after_sync();
           issue_pv(next_pv);
           ++next_pv;
@@ -448,7 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     }
   } else if (warp >= 4 && warp < 12) {
     // ======================= softmax (two warpgroups, alternating items) =======================
-    const int wg = (warp - 4) >> 2;      // warpgroup: handles items i with i % NP == wg
+    // With one S slot a second warpgroup would wait on a barrier phase two ahead of the
+    // last one it saw, which a parity wait cannot tell apart: one warpgroup then.
+    constexpr int kWG = NP >= 2 ? 2 : 1;
+    const int wg = (warp - 4) >> 2;      // warpgroup: handles items i with i % kWG == wg
     const int t = (tid - 128) & 127;     // tile row == TMEM lane
     const int wq = warp & 3;             // TMEM lane quadrant
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
@@ -496,13 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     };
     float sh_next = row_score(wg);
     bool synced_own = false;
-    for (int i = wg; i < n_items && wg < NP; i += NP) {
+    for (int i = wg; i < n_items && wg < kWG; i += kWG) {
       const int b = i % NP;
       int c, t0, n_rows;
       bool own;
       item_rows(s_items[i], c, own, t0, n_rows);
       const float sh = sh_next;
-      sh_next = row_score(i + NP);
+      sh_next = row_score(i + kWG);
       if (!own && !synced_own) {
         named_bar(1, 256);  // every row's (M, 1/Z') is final once the own items are done
         synced_own = true;
@@ -639,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         tc::tmem_wait_ld();
       }
       for (int i = 0; i < n_items; ++i) {
-        const int o = i & 1;
+        const int o = i % NO;
         if (ok && cur.warp_ok) tc::tmem_ld32(tO0 + o * 64 + 32 + lane_off, vb);
         if (ok && cur.row_ok) add32(va, cur, 0);
         tc::tmem_wait_ld();
@@ -647,10 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         mbar_arrive(tc::smem_u32(&bar_ofree[o]));  // item i has left TMEM
         Geo nxt{};
         if (i + 1 < n_items) {
-          ok = __all_sync(0xffffffffu, ok && wait(&bar_ofull[(i + 1) & 1], (uint32_t)(((i + 1) >> 1) & 1)));
+          ok = __all_sync(0xffffffffu, ok && wait(&bar_ofull[(i + 1) % NO], (uint32_t)(((i + 1) / NO) & 1)));
           tc::fence_after_sync();
           nxt = geo(i + 1);
-          if (ok && nxt.warp_ok) tc::tmem_ld32(tO0 + ((i + 1) & 1) * 64 + lane_off, va);
+          if (ok && nxt.warp_ok) tc::tmem_ld32(tO0 + ((i + 1) % NO) * 64 + lane_off, va);
         }
         if (ok && cur.row_ok) add32(vb, cur, 32);
         tc::tmem_wait_ld();
@@ -659,8 +667,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       }
     } else {
       for (int i = 0; i < n_items; ++i) {
-        const int o = i & 1;
-        const bool ok = __all_sync(0xffffffffu, wait(&bar_ofull[o], (uint32_t)((i >> 1) & 1)));
+        const int o = i % NO;
+        const bool ok = __all_sync(0xffffffffu, wait(&bar_ofull[o], (uint32_t)((i / NO) & 1)));
         tc::fence_after_sync();
         const Geo g = geo(i);
         if (ok && g.warp_ok) {
