@@ -2,13 +2,13 @@
 // applied to the newest query of each sequence).  Two HBM-bound kernels,
 // chained with programmatic dependent launch:
 //
-// 1. decode_scan_kernel -- grid (sequence, KV head, range of kScanChunks
-//    candidate chunks).  Each CTA scores its range against the cached
-//    summaries (q . kbar * scale + H, GQA max over the group's heads), sorts
-//    the range's packed keys (bitonic, shared memory) and writes its best K.
-//    The last CTA of the (sequence, KV head) -- an atomic ticket; no CTA waits
-//    on another -- merges the lists into the final Top-K and writes each
-//    head's own score of the selected chunks.
+// 1. decode_scan_kernel -- grid (sequence, range of candidate chunks).  Each CTA
+//    reads the cached summaries of its range page by page, all heads at once (a
+//    page's [h][d] fp32 block is contiguous), scores them (q . kbar * scale + H, GQA
+//    max over the group's heads) and, one warp per KV head, sorts the range's keys
+//    and writes its best K.  The last CTA of the sequence -- an atomic ticket; no
+//    CTA waits on another -- merges the ranges' lists into the final Top-K and
+//    writes each head's own score of the selected chunks.
 // 2. decode_attend_kernel -- one warp per chunk (own chunk or one Top-K slot),
 //    all G heads sharing each K/V load, K and V staged in shared memory with
 //    cp.async.  The own chunk does not depend on the selection and is
@@ -25,192 +25,331 @@ namespace hils {
 
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kScanChunks = 128;   // candidate chunks per scan CTA (power of two)
-constexpr int kMergeCap = 2048;    // keys the merging CTA sorts at once (power of two)
+constexpr int kMaxRange = 256;          // candidate chunks per scan CTA, at most ...
+constexpr int kMinRange = 16;           // ... and at least
+constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B200
+constexpr int kMergeN = 256;            // keys one warp sorts at once in the fallback merge
+constexpr int kMergeBuf = 1536;         // keys per warp staged in shared memory for the tournament merge
 
 // chunks (warps) per attend CTA: K and V of a chunk are staged per warp, so wide rows get fewer warps
 template <typename T, int D>
 __host__ __device__ constexpr int att_warps() { return sizeof(T) * D <= 256 ? 4 : 2; }
 
-int decode_splits(int max_chunks) { return max(1, (max_chunks + kScanChunks - 1) / kScanChunks); }
+// Ranges per sequence: ranges of kMinRange..kMaxRange chunks, enough of them for about
+// kScanCtasTarget CTAs over the batch.  A pure function of the shape, so the workspace
+// layout and the launch agree.
+int decode_splits(int batch, int max_chunks) {
+  const int lo = (max_chunks + kMaxRange - 1) / kMaxRange;
+  const int hi = max(1, (max_chunks + kMinRange - 1) / kMinRange);
+  const int want = (kScanCtasTarget + max(1, batch) - 1) / max(1, batch);
+  return max(lo, min(hi, want));
+}
+bool decode_supported(int h, int d) { return h * d <= 8 * kScanThreads * 4; }
+constexpr int kMaxListsPerLane = 4;
+
+// The tournament merge stages every range's list of the KV head in shared memory.
+__host__ __device__ inline bool merge_in_smem(int nsplit, int K) {
+  return nsplit <= 32 * kMaxListsPerLane && nsplit * K <= kMergeBuf;
+}
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// Descending bitonic sort of keys[0..n), n a power of two; the whole block calls it.
-template <int THREADS>
-__device__ void block_sort_desc(unsigned long long* keys, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// Descending bitonic sort of the warp's 32*E keys; element i lives in lane i / E,
+// register i % E.  All 32 lanes call it.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(unsigned long long (&v)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += THREADS) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long x = keys[i], y = keys[ixj];
-          const bool desc = (i & k) == 0;
-          if (desc ? (x < y) : (x > y)) {
-            keys[i] = y;
-            keys[ixj] = x;
+      if (j >= E) {  // partner in lane ^ (j / E), same register
+        const int lj = j / E;
+        const bool lower = (lane & lj) == 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const bool desc = ((lane * E + e) & k) == 0;
+          const unsigned long long o = shfl_xor_u64(v[e], lj);
+          const bool keep_max = lower == desc;
+          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+      } else {  // partner in this lane, register e ^ j
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if ((e ^ j) > e) {
+            const bool desc = ((lane * E + e) & k) == 0;
+            const unsigned long long x = v[e], y = v[e ^ j];
+            const bool sw = desc ? x < y : x > y;
+            v[e] = sw ? y : x;
+            v[e ^ j] = sw ? x : y;
           }
         }
       }
-      __syncthreads();
     }
   }
 }
-
-__device__ __forceinline__ int pow2_ceil(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a) {
-  constexpr int LPR = D / 4;              // lanes per summary row (one float4 each)
-  constexpr int RPW = 32 / LPR;           // rows per warp step
-  __shared__ unsigned long long s_keys[kMergeCap];
-  __shared__ float s_score[kScanChunks * G];
-  __shared__ int s_page[kScanChunks];
-  __shared__ int s_sel[kMaxTopK];
-  __shared__ int s_last;
-
-  pdl_launch_dependents();  // the attend grid may start its selection-independent prologue
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  // CTA order (sequence, range, KV head): the CTAs of all heads of one range run
-  // together, so each page's summary block is read from DRAM in one burst
-  const int gi = blockIdx.x % a.g;
-  const int split = (blockIdx.x / a.g) % a.nsplit;
-  const int bi = blockIdx.x / (a.nsplit * a.g);
-  const int K = a.top_k;
-  const int c_lo = split * kScanChunks;
-  const int32_t* bt = a.block_table + (size_t)bi * a.max_chunks;
-  // block-table slice and the query are loaded alongside the sequence length
-  for (int x = t; x < kScanChunks; x += kScanThreads)
-    s_page[x] = c_lo + x < a.max_chunks ? bt[c_lo + x] : -1;
-  const int sub = lane % LPR;
-  float4 qv[G];
+// Top-K of one KV head over this CTA's range: the key of chunk j is the max over the
+// group's heads of s_score[j][head] (a NaN, from a bad page, makes the key 0).  Writes
+// the K best keys (0 where the range has fewer) in descending order.
+template <int E, int G>
+__device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, int nc, int c_lo, int K,
+                                           unsigned long long* out) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long v[E];
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh)
-    qv[hh] = load4(static_cast<const T*>(a.q) + ((size_t)bi * a.h + gi * G + hh) * D + sub * 4);
-  const int L = a.seq_lens[bi];
-  const int own = L > 0 ? (L - 1) / kChunk : 0;
-  const int n_cand = min(own, a.max_chunks);
-  const int nc = max(0, min(n_cand, c_lo + kScanChunks) - c_lo);
-  __syncthreads();
-
-  // score rows (chunk, head): every warp issues kBatch loads before reducing them
-  constexpr int kBatch = 8;
-  const int n_rows = nc * G;
-  const int step = kScanWarps * RPW;
-  for (int r0 = warp * RPW; r0 < n_rows; r0 += step * kBatch) {
-    float4 kv[kBatch];
-    int pg[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int r = r0 + u * step + lane / LPR;
-      pg[u] = -1;
-      kv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < n_rows) {
-        const int p = s_page[r / G];
-        if (p >= 0 && p < a.n_pages) {
-          pg[u] = p;
-          kv[u] = __ldg(reinterpret_cast<const float4*>(a.kbar_pages + ((size_t)p * a.h + gi * G + r % G) * D + sub * 4));
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int r = r0 + u * step + lane / LPR;
-      const int hh = r % G;
-      float4 q = qv[0];
-#pragma unroll
-      for (int x = 1; x < G; ++x)
-        if (hh == x) q = qv[x];
-      float dot = fmaf(q.x, kv[u].x, fmaf(q.y, kv[u].y, fmaf(q.z, kv[u].z, q.w * kv[u].w)));
-#pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      if (r < n_rows && sub == 0) {
-        const int p = pg[u];
-        if (p < 0) set_error(a.err, kErrBadPage);
-        s_score[r] = p >= 0 ? fmaf(dot, a.scale, __ldg(a.hbias_pages + (size_t)p * a.h + gi * G + hh)) : NAN;
-      }
-    }
-  }
-  __syncthreads();
-  for (int cl = t; cl < kScanChunks; cl += kScanThreads) {
+  for (int e = 0; e < E; ++e) {
+    const int j = e * 32 + lane;  // any placement works: the keys are sorted next
     unsigned long long key = 0;
-    if (cl < nc) {
+    if (j < nc) {
       float best = -INFINITY;
       bool bad = false;
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        const float v = s_score[cl * G + hh];
-        bad |= (v != v);
-        best = fmaxf(best, v);
+        const float x = s_score[(size_t)j * H + gi * G + hh];
+        bad |= x != x;
+        best = fmaxf(best, x);
       }
-      key = bad ? 0ull : pack_key(best, c_lo + cl);
+      key = bad ? 0ull : pack_key(best, c_lo + j);
     }
-    s_keys[cl] = key;
+    v[e] = key;
+  }
+  warp_sort_desc<E>(v);
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane * E + e;
+    if (i < K) out[i] = v[e];
+  }
+  for (int i = 32 * E + lane; i < K; i += 32) out[i] = 0ull;
+}
+
+// Scan: CTA per (sequence, range of chunks), all heads.  A page's summaries of all
+// heads, [h][d] fp32, are one contiguous block; thread t holds float4 t + 256 k of it
+// (FPT per thread), so each page is read with fully coalesced 16-byte loads, PB pages
+// in flight per thread.  Per (chunk, head) the dot with q is reduced over the d/4
+// lanes of the head row, scaled and biased by H into shared memory; then one warp per
+// KV head sorts the range's keys and writes its best K.  The last CTA of the sequence
+// (atomic ticket; no CTA waits on another) merges the ranges' lists.
+template <typename T, int D, int G, int FPT>
+__global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) float s_score[];  // [range][h]; reused by the merge
+  __shared__ int s_page[kMaxRange];
+  __shared__ int s_last;
+  constexpr int QPR = D / 4;                     // float4 per head row
+  constexpr int PB = FPT >= 8 ? 1 : 8 / FPT;     // pages per batch (two batches in flight)
+
+  pdl_launch_dependents();  // the attend grid may start its selection-independent prologue
+  const int t = threadIdx.x, warp = t >> 5;
+  const int split = blockIdx.x % a.nsplit;
+  const int bi = blockIdx.x / a.nsplit;
+  const int H = a.h, K = a.top_k, R = a.range;
+  const int c_lo = split * R;
+  const int32_t* bt = a.block_table + (size_t)bi * a.max_chunks;
+  const int L = a.seq_lens[bi];
+  const int own = L > 0 ? (L - 1) / kChunk : 0;
+  const int n_cand = min(own, a.max_chunks);
+  const int nc = max(0, min(n_cand, c_lo + R) - c_lo);
+  for (int x = t; x < nc; x += kScanThreads) s_page[x] = bt[c_lo + x];
+  const int F = H * QPR;  // float4 per page block
+  float4 qv[FPT];
+#pragma unroll
+  for (int k = 0; k < FPT; ++k) {
+    const int f = t + k * kScanThreads;
+    qv[k] = f < F ? load4(static_cast<const T*>(a.q) + ((size_t)bi * H + f / QPR) * D + (f % QPR) * 4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
-  block_sort_desc<kScanThreads>(s_keys, kScanChunks);
-  unsigned long long* part = a.part_keys + (((size_t)bi * a.g + gi) * a.nsplit + split) * K;
-  for (int s = t; s < K; s += kScanThreads) part[s] = s_keys[s];
+
+  // Pages are processed in batches of PB, double-buffered: the next batch's loads are
+  // in flight while the current one is reduced.
+  const float4* kb4 = reinterpret_cast<const float4*>(a.kbar_pages);
+  struct Batch {
+    float4 kv[PB][FPT];
+    float hv[PB][FPT];  // H of the lane's head (read by the lane that writes the score)
+    int pg[PB];
+  };
+  auto load = [&](Batch& B, int j0) {
+#pragma unroll
+    for (int u = 0; u < PB; ++u) {
+      const int j = j0 + u;
+      B.pg[u] = j < nc ? s_page[j] : -1;
+      const bool ok = B.pg[u] >= 0 && B.pg[u] < a.n_pages;
+#pragma unroll
+      for (int k = 0; k < FPT; ++k) {
+        const int f = t + k * kScanThreads;
+        B.kv[u][k] = ok && f < F ? __ldg(kb4 + (size_t)B.pg[u] * F + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        B.hv[u][k] = ok && f < F && f % QPR == 0 ? __ldg(a.hbias_pages + (size_t)B.pg[u] * H + f / QPR) : 0.f;
+      }
+    }
+  };
+  auto reduce = [&](const Batch& B, int j0) {
+#pragma unroll
+    for (int u = 0; u < PB; ++u) {
+      const int j = j0 + u;
+#pragma unroll
+      for (int k = 0; k < FPT; ++k) {
+        const int f = t + k * kScanThreads;
+        const float4 kv = B.kv[u][k];
+        float dot = fmaf(qv[k].x, kv.x, fmaf(qv[k].y, kv.y, fmaf(qv[k].z, kv.z, qv[k].w * kv.w)));
+#pragma unroll
+        for (int o = QPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (j < nc && f < F && f % QPR == 0) {
+          const int head = f / QPR, p = B.pg[u];
+          float sc = NAN;
+          if (p >= 0 && p < a.n_pages) sc = fmaf(dot, a.scale, B.hv[u][k]);
+          else set_error(a.err, kErrBadPage);
+          s_score[(size_t)j * H + head] = sc;
+        }
+      }
+    }
+  };
+  Batch b0, b1;
+  load(b0, 0);
+  for (int j0 = 0; j0 < nc; j0 += 2 * PB) {
+    load(b1, j0 + PB);
+    reduce(b0, j0);
+    load(b0, j0 + 2 * PB);
+    reduce(b1, j0 + PB);
+  }
+  __syncthreads();
+
+  // per KV head: this range's best K
+  const int E = nc <= 32 ? 1 : nc <= 64 ? 2 : nc <= 128 ? 4 : 8;
+  for (int gi = warp; gi < a.g; gi += kScanWarps) {
+    unsigned long long* part = a.part_keys + (((size_t)bi * a.g + gi) * a.nsplit + split) * K;
+    switch (E) {
+      case 1: range_topk<1, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      case 2: range_topk<2, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      case 4: range_topk<4, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      default: range_topk<8, G>(s_score, H, gi, nc, c_lo, K, part); break;
+    }
+  }
   __threadfence();
   __syncthreads();
-  if (t == 0) s_last = atomicAdd(a.scan_ticket + (size_t)bi * a.g + gi, 1u) == (unsigned)(a.nsplit - 1);
+  if (t == 0) s_last = atomicAdd(a.scan_ticket + (size_t)bi * a.g, 1u) == (unsigned)(a.nsplit - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
 
-  // ---- last CTA: merge the per-range lists (running best K + next slice) ----
-  const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * a.nsplit * K;
+  // ---- last CTA of the sequence: per KV head, merge the ranges' lists ----
+  const int lane = t & 31;
   const int n_all = a.nsplit * K;
-  for (int x = t; x < K; x += kScanThreads) s_keys[x] = 0;
-  for (int start = 0; start < n_all; start += kMergeCap - K) {
-    const int take = min(kMergeCap - K, n_all - start);
-    const int n2 = pow2_ceil(K + take);
-    __syncthreads();
-    for (int x = t; x < n2 - K; x += kScanThreads) s_keys[K + x] = x < take ? __ldcg(parts + start + x) : 0ull;
-    __syncthreads();
-    block_sort_desc<kScanThreads>(s_keys, n2);
-  }
-  for (int s = t; s < K; s += kScanThreads) {
-    const unsigned long long key = s_keys[s];
-    s_sel[s] = key ? key_chunk(key) : -1;
-  }
-  __syncthreads();
-  for (int s = t; s < K; s += kScanThreads) {
-    const int c = s_sel[s];
-    a.idx[((size_t)bi * a.g + gi) * K + s] = c;
-    a.sel_page[((size_t)bi * a.g + gi) * K + s] = c >= 0 ? bt[c] : -1;
-  }
-  if constexpr (G == 1) {
-    // the selection key is the head's own score
-    for (int s = t; s < K; s += kScanThreads) {
-      const unsigned long long key = s_keys[s];
-      a.ssel[((size_t)bi * a.h + gi) * K + s] = key ? unorderable((uint32_t)(key >> 32)) : -INFINITY;
+  // the selected keys of slots lane and lane + 32, in descending order (0: empty)
+  auto emit = [&](int gi, unsigned long long k0, unsigned long long k1) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int s = lane + 32 * r;
+      const unsigned long long key = r ? k1 : k0;
+      if (s < K) {
+        const int c = key ? (int)key_chunk(key) : -1;
+        a.idx[((size_t)bi * a.g + gi) * K + s] = c;
+        a.sel_page[((size_t)bi * a.g + gi) * K + s] = c >= 0 ? bt[c] : -1;
+        // G = 1: the selection key is the head's own score
+        if (G == 1) a.ssel[((size_t)bi * a.h + gi) * K + s] = key ? unorderable((uint32_t)(key >> 32)) : -INFINITY;
+      }
+    }
+  };
+  if (merge_in_smem(a.nsplit, K)) {
+    // tournament: the lists are sorted, so each step is a warp max over the lists' heads
+    // (keys are unique: they carry the chunk index); lane l follows lists l, l + 32, ...
+    unsigned long long* s_m = reinterpret_cast<unsigned long long*>(s_score) + (size_t)warp * n_all;
+    for (int gi = warp; gi < a.g; gi += kScanWarps) {
+      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
+      __syncwarp();
+      for (int x = lane; x < n_all; x += 32) s_m[x] = __ldcg(parts + x);
+      __syncwarp();
+      int pos[kMaxListsPerLane];
+      unsigned long long head[kMaxListsPerLane];
+#pragma unroll
+      for (int m = 0; m < kMaxListsPerLane; ++m) {
+        const int l = lane + 32 * m;
+        pos[m] = 0;
+        head[m] = l < a.nsplit ? s_m[(size_t)l * K] : 0ull;
+      }
+      unsigned long long res0 = 0ull, res1 = 0ull;
+      for (int s = 0; s < K; ++s) {
+        unsigned long long lb = head[0];
+#pragma unroll
+        for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
+        unsigned long long wb = lb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = shfl_xor_u64(wb, o);
+          wb = y > wb ? y : wb;
+        }
+        if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
+#pragma unroll
+        for (int m = 0; m < kMaxListsPerLane; ++m) {
+          if (head[m] == wb) {  // this lane's list m holds the winner: advance it
+            ++pos[m];
+            head[m] = pos[m] < K ? s_m[(size_t)(lane + 32 * m) * K + pos[m]] : 0ull;
+          }
+        }
+        if ((s & 31) == lane) {
+          if (s < 32) res0 = wb;
+          else res1 = wb;
+        }
+      }
+      emit(gi, res0, res1);
     }
   } else {
-    // each head's own score of the selected chunks: one warp per (slot, head)
-    for (int x = warp; x < K * G; x += kScanWarps) {
-      const int s = x / G, hh = x % G;
-      const int c = s_sel[s];
+    // running best K + the next slice of keys, sorted by the warp
+    for (int gi = warp; gi < a.g; gi += kScanWarps) {
+      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
+      constexpr int ME = kMergeN / 32;
+      unsigned long long v[ME];
+#pragma unroll
+      for (int e = 0; e < ME; ++e) v[e] = 0ull;
+      for (int start = 0; start < n_all; start += kMergeN - K) {
+        const int take = min(kMergeN - K, n_all - start);
+#pragma unroll
+        for (int e = 0; e < ME; ++e) {
+          const int i = lane * ME + e;
+          if (i >= K) v[e] = i - K < take ? __ldcg(parts + start + i - K) : 0ull;
+        }
+        warp_sort_desc<ME>(v);
+      }
+      // slot s sits in lane s / ME, register s % ME: move slots lane and lane + 32 here
+      unsigned long long k0 = 0ull, k1 = 0ull;
+#pragma unroll
+      for (int e = 0; e < ME; ++e) {
+        const unsigned long long x0 = __shfl_sync(0xffffffffu, (uint32_t)v[e], lane / ME) |
+                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), lane / ME) << 32);
+        const unsigned long long x1 = __shfl_sync(0xffffffffu, (uint32_t)v[e], (lane + 32) / ME) |
+                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), (lane + 32) / ME) << 32);
+        if (lane % ME == e) k0 = x0;
+        if ((lane + 32) % ME == e) k1 = x1;
+      }
+      emit(gi, k0, k1);
+    }
+  }
+  if constexpr (G > 1) {
+    __syncthreads();  // the selection written above is read back below
+    // each head's own score of the selected chunks: one warp per (KV head, slot, head)
+    for (int x = warp; x < a.g * K * G; x += kScanWarps) {
+      const int gi = x / (K * G), s = (x / G) % K, hh = x % G;
+      const int c = a.idx[((size_t)bi * a.g + gi) * K + s];
       float sc = -INFINITY;
       if (c >= 0) {
         const int p = bt[c];
-        const float* kb = a.kbar_pages + ((size_t)p * a.h + gi * G + hh) * D;
-        const T* qr = static_cast<const T*>(a.q) + ((size_t)bi * a.h + gi * G + hh) * D;
+        const float* kb = a.kbar_pages + ((size_t)p * H + gi * G + hh) * D;
+        const T* qr = static_cast<const T*>(a.q) + ((size_t)bi * H + gi * G + hh) * D;
         float acc = 0.f;
 #pragma unroll
         for (int e = lane; e < D; e += 32) acc = fmaf(to_f(qr[e]), __ldg(kb + e), acc);
         acc = warp_sum(acc);
-        sc = fmaf(acc, a.scale, __ldg(a.hbias_pages + (size_t)p * a.h + gi * G + hh));
+        sc = fmaf(acc, a.scale, __ldg(a.hbias_pages + (size_t)p * H + gi * G + hh));
       }
-      if (lane == 0) a.ssel[((size_t)bi * a.h + gi * G + hh) * K + s] = sc;
+      if (lane == 0) a.ssel[((size_t)bi * H + gi * G + hh) * K + s] = sc;
     }
   }
-  if (t == 0) a.scan_ticket[(size_t)bi * a.g + gi] = 0;
+  if (t == 0) a.scan_ticket[(size_t)bi * a.g] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -396,13 +535,29 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
   if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
 }
 
+template <typename T, int D, int G, int FPT>
+static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
+  size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores; reused by the merge
+  if (merge_in_smem(a.nsplit, a.top_k)) smem = max(smem, (size_t)kScanWarps * a.nsplit * a.top_k * 8);
+  cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, FPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_scan_kernel<T, D, G, FPT><<<(unsigned)a.b * a.nsplit, kScanThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int G>
 static cudaError_t launch_decode(DecodeArgs a, cudaStream_t st) {
   const unsigned bg = (unsigned)a.b * a.g;
   if (bg == 0) return cudaSuccess;
+  if (!decode_supported(a.h, D)) return cudaErrorInvalidValue;
   if (a.top_k > 0) {
-    decode_scan_kernel<T, D, G><<<bg * a.nsplit, kScanThreads, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    const int f4 = a.h * D / 4;  // float4 per page of summaries
+    const int fpt = (f4 + kScanThreads - 1) / kScanThreads;
+    cudaError_t e = fpt <= 1 ? launch_scan<T, D, G, 1>(a, st)
+                  : fpt <= 2 ? launch_scan<T, D, G, 2>(a, st)
+                  : fpt <= 4 ? launch_scan<T, D, G, 4>(a, st)
+                             : launch_scan<T, D, G, 8>(a, st);
     if (e != cudaSuccess) return e;
   }
   constexpr int AW = att_warps<T, D>();
@@ -438,7 +593,8 @@ static cudaError_t decode_by_group(const DecodeArgs& a, cudaStream_t st) {
 }
 
 cudaError_t run_decode(DecodeArgs a, cudaStream_t st) {
-  a.nsplit = decode_splits(a.max_chunks);
+  a.nsplit = decode_splits(a.b, a.max_chunks);
+  a.range = (a.max_chunks + a.nsplit - 1) / a.nsplit;
   if (a.bf16) return a.d == 64 ? decode_by_group<__nv_bfloat16, 64>(a, st) : decode_by_group<__nv_bfloat16, 128>(a, st);
   return a.d == 64 ? decode_by_group<float, 64>(a, st) : decode_by_group<float, 128>(a, st);
 }

@@ -63,7 +63,7 @@ DecodeLayout decode_layout(const hils_shape* s) {
   const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k, d = s->head_dim;
   const size_t G = h / g;
   const int cmax = (s->seq_len + s->chunk - 1) / s->chunk;
-  const size_t nsplit = hils::decode_splits(cmax);
+  const size_t nsplit = hils::decode_splits(s->batch, cmax);
   DecodeLayout L;
   size_t off = kHeader;
   L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
@@ -253,6 +253,7 @@ hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages,
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if (s->batch == 0) return HILS_OK;
+  if (!hils::decode_supported(s->heads_q, s->head_dim)) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
@@ -329,7 +330,7 @@ StaticLayout static_decode_layout(const hils_shape* s) {
   const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, K = s->top_k, d = s->head_dim;
   const size_t G = h / g;
   const int cmax = (s->seq_len + s->chunk - 1) / s->chunk;
-  const size_t nsplit = hils::decode_splits(cmax);
+  const size_t nsplit = hils::decode_splits(s->batch, cmax);
   StaticLayout L;
   size_t off = kHeader;
   L.scan_ticket = off; off += kStaticTicketSlots * 4;
@@ -375,6 +376,7 @@ hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if (s->batch == 0) return HILS_OK;
+  if (!hils::decode_supported(s->heads_q, s->head_dim)) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)

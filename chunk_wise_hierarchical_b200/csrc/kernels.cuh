@@ -52,17 +52,18 @@ struct DecodeArgs {
   int32_t* idx;                // [b,g,K]
   int32_t* sel_page;           // [b,g,K] page of each selected chunk
   float* ssel;                 // [b,h,K]
-  unsigned long long* part_keys;  // [b,g,nsplit,K]
+  unsigned long long* part_keys;  // [b,g,nsplit,K] per-range Top-K lists
   float* part_att;             // [b,g,K+1,G,d+2]
-  unsigned* scan_ticket;       // [b,g]
+  unsigned* scan_ticket;       // [b,g] (the scan uses entry (b, 0))
   unsigned* att_ticket;        // [b,g]
   unsigned* err;
   int b, h, g, d, top_k, max_chunks, n_pages;
-  int nsplit, att_ctas;        // set by the launcher
+  int nsplit, range, att_ctas; // set by the launcher: scan ranges per sequence, chunks per range
   float scale;
   bool bf16;
 };
-int decode_splits(int max_chunks);
+int decode_splits(int batch, int max_chunks);
+bool decode_supported(int h, int d);  // the scan holds a page's summaries of all heads: h * d <= 8192
 cudaError_t run_decode(DecodeArgs a, cudaStream_t st);
 
 // Row-wise attention + fusion (one warp per query and KV group).
