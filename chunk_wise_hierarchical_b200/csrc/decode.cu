@@ -29,7 +29,6 @@ constexpr int kMaxRange = 256;          // candidate chunks per scan CTA, at mos
 constexpr int kMinRange = 16;           // ... and at least
 constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B200
 constexpr int kMergeN = 256;            // keys one warp sorts at once in the fallback merge
-constexpr int kMergeBuf = 1536;         // keys per warp staged in shared memory for the tournament merge
 
 // chunks (warps) per attend CTA: K and V of a chunk are staged per warp, so wide rows get fewer warps
 template <typename T, int D>
@@ -47,10 +46,6 @@ int decode_splits(int batch, int max_chunks) {
 bool decode_supported(int h, int d) { return h * d <= 8 * kScanThreads * 4; }
 constexpr int kMaxListsPerLane = 4;
 
-// The tournament merge stages every range's list of the KV head in shared memory.
-__host__ __device__ inline bool merge_in_smem(int nsplit, int K) {
-  return nsplit <= 32 * kMaxListsPerLane && nsplit * K <= kMergeBuf;
-}
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -136,13 +131,15 @@ __device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, 
 // lanes of the head row, scaled and biased by H into shared memory; then one warp per
 // KV head sorts the range's keys and writes its best K.  The last CTA of the sequence
 // (atomic ticket; no CTA waits on another) merges the ranges' lists.
+// Four CTAs per SM (64 registers a thread): a page gather's bandwidth grows with the
+// warps resident on the SM far more than with the loads each warp has in flight.
 template <typename T, int D, int G, int FPT>
-__global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) float s_score[];  // [range][h]; reused by the merge
   __shared__ int s_page[kMaxRange];
   __shared__ int s_last;
   constexpr int QPR = D / 4;                     // float4 per head row
-  constexpr int PB = FPT >= 8 ? 1 : 8 / FPT;     // pages per batch (two batches in flight)
+  constexpr int PB = FPT >= 8 ? 1 : 8 / FPT;     // pages per batch of loads
 
   pdl_launch_dependents();  // the attend grid may start its selection-independent prologue
   const int t = threadIdx.x, warp = t >> 5;
@@ -166,8 +163,8 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a)
   }
   __syncthreads();
 
-  // Pages are processed in batches of PB, double-buffered: the next batch's loads are
-  // in flight while the current one is reduced.
+  // Pages are processed in batches of PB: the batch's loads are all in flight before
+  // the first is reduced.
   const float4* kb4 = reinterpret_cast<const float4*>(a.kbar_pages);
   struct Batch {
     float4 kv[PB][FPT];
@@ -209,13 +206,10 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a)
       }
     }
   };
-  Batch b0, b1;
-  load(b0, 0);
-  for (int j0 = 0; j0 < nc; j0 += 2 * PB) {
-    load(b1, j0 + PB);
-    reduce(b0, j0);
-    load(b0, j0 + 2 * PB);
-    reduce(b1, j0 + PB);
+  for (int j0 = 0; j0 < nc; j0 += PB) {
+    Batch bt_;
+    load(bt_, j0);
+    reduce(bt_, j0);
   }
   __syncthreads();
 
@@ -255,22 +249,22 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a)
       }
     }
   };
-  if (merge_in_smem(a.nsplit, K)) {
+  if (a.nsplit <= 32 * kMaxListsPerLane) {
     // tournament: the lists are sorted, so each step is a warp max over the lists' heads
-    // (keys are unique: they carry the chunk index); lane l follows lists l, l + 32, ...
-    unsigned long long* s_m = reinterpret_cast<unsigned long long*>(s_score) + (size_t)warp * n_all;
+    // (keys are unique: they carry the chunk index).  Lane l follows lists l, l + 32, ...
+    // straight from global memory, holding each list's head and the key after it, and
+    // fetching the next one as soon as a head is taken.
     for (int gi = warp; gi < a.g; gi += kScanWarps) {
       const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
-      __syncwarp();
-      for (int x = lane; x < n_all; x += 32) s_m[x] = __ldcg(parts + x);
-      __syncwarp();
       int pos[kMaxListsPerLane];
-      unsigned long long head[kMaxListsPerLane];
+      unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
 #pragma unroll
       for (int m = 0; m < kMaxListsPerLane; ++m) {
         const int l = lane + 32 * m;
+        const bool live = l < a.nsplit;
         pos[m] = 0;
-        head[m] = l < a.nsplit ? s_m[(size_t)l * K] : 0ull;
+        head[m] = live ? __ldcg(parts + (size_t)l * K) : 0ull;
+        next[m] = live && K > 1 ? __ldcg(parts + (size_t)l * K + 1) : 0ull;
       }
       unsigned long long res0 = 0ull, res1 = 0ull;
       for (int s = 0; s < K; ++s) {
@@ -288,7 +282,8 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(DecodeArgs a)
         for (int m = 0; m < kMaxListsPerLane; ++m) {
           if (head[m] == wb) {  // this lane's list m holds the winner: advance it
             ++pos[m];
-            head[m] = pos[m] < K ? s_m[(size_t)(lane + 32 * m) * K + pos[m]] : 0ull;
+            head[m] = next[m];
+            next[m] = pos[m] + 1 < K ? __ldcg(parts + (size_t)(lane + 32 * m) * K + pos[m] + 1) : 0ull;
           }
         }
         if ((s & 31) == lane) {
@@ -537,8 +532,7 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
 
 template <typename T, int D, int G, int FPT>
 static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
-  size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores; reused by the merge
-  if (merge_in_smem(a.nsplit, a.top_k)) smem = max(smem, (size_t)kScanWarps * a.nsplit * a.top_k * 8);
+  const size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores
   cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, FPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
