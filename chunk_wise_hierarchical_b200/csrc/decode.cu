@@ -30,9 +30,6 @@ constexpr int kMinRange = 16;           // ... and at least
 constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B200
 constexpr int kMergeN = 256;            // keys one warp sorts at once in the fallback merge
 
-// chunks (warps) per attend CTA: K and V of a chunk are staged per warp, so wide rows get fewer warps
-template <typename T, int D>
-__host__ __device__ constexpr int att_warps() { return sizeof(T) * D <= 256 ? 4 : 2; }
 
 // Ranges per sequence: ranges of kMinRange..kMaxRange chunks, enough of them for about
 // kScanCtasTarget CTAs over the batch.  A pure function of the shape, so the workspace
@@ -348,15 +345,61 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
 }
 
 // ---------------------------------------------------------------------------
+// Attention: one warp per half chunk (32 keys) of the own chunk or of a Top-K slot,
+// all G heads sharing each K/V load.  Lanes own keys for Q.K (each reads its key row)
+// and output columns for P.V (V rows are read across the lanes); nothing is staged,
+// so many warps fit per SM.  Each warp writes its half's (max, sum, unnormalised
+// output) per head; the last CTA of the (sequence, KV head) combines the halves of
+// each chunk and fuses the chunks with the inter-chunk softmax of notes section 5.3
+// (own chunk at its exact log-mass).
+constexpr int kAttWarps = 4;
+
+// Raw register types for one lane's share of a V row (CPL elements of T).
+template <int BYTES> struct RawT;
+template <> struct RawT<4> { using type = uint32_t; };
+template <> struct RawT<8> { using type = uint2; };
+template <> struct RawT<16> { using type = uint4; };
+
+template <typename T, int CPL>
+__device__ __forceinline__ void raw_to_f(const typename RawT<CPL * sizeof(T)>::type& r, float (&f)[CPL]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&r);
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < CPL / 2; ++i) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) f[i] = __uint_as_float(w[i]);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_row16(const T* src, float (&f)[16 / sizeof(T)]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(h[i]);
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  } else {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+}
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(DecodeArgs a) {
-  constexpr int kAttWarps = att_warps<T, D>();
-  constexpr int CPL = D / 32;                 // output columns per lane (adjacent)
-  constexpr int RS = D + 16 / (int)sizeof(T); // padded shared row (elements): rows hit different banks
-  extern __shared__ __align__(16) unsigned char dyn[];
-  T* s_kv = reinterpret_cast<T*>(dyn);        // [warps][2][64][RS]
+__global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArgs a) {
+  constexpr int CPL = D / 32;                  // output columns per lane (adjacent)
+  constexpr int EPP = 16 / (int)sizeof(T);     // elements per 16-byte piece
+  constexpr int PPR = D / EPP;                 // pieces per key row
   __shared__ __align__(16) float qS[G][D];
-  __shared__ float s_w[kAttWarps][kMaxTopK + 1];
+  __shared__ float s_w[G][2 * (kMaxTopK + 1)];  // fusion weight of each half chunk, per head
   __shared__ int s_last;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -365,7 +408,7 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
   const int gi = (blockIdx.x / ngrp) % a.g;
   const int bi = blockIdx.x / (ngrp * a.g);
   const int K = a.top_k;
-  const int n_items = K + 1;                  // item 0: own chunk; item s >= 1: Top-K slot s-1
+  const int n_items = 2 * (K + 1);             // item 2s + hf: slot s (0 own, s >= 1 Top-K s-1), half hf
   const size_t part_stride = (size_t)G * (D + 2);
   float* part = a.part_att + ((size_t)bi * a.g + gi) * (size_t)n_items * part_stride;
   const int L = a.seq_lens[bi];
@@ -373,95 +416,103 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
     qS[x / D][x % D] = to_f(static_cast<const T*>(a.q)[((size_t)bi * a.h + gi * G) * D + x]);
   __syncthreads();
 
-  T* sk = s_kv + (size_t)warp * 2 * kChunk * RS;
-  T* sv = sk + (size_t)kChunk * RS;
   const int item = grp_i * kAttWarps + warp;
-  // one chunk: returns false if absent
+  const int hf = item & 1;
   auto run_item = [&](int c, int p, int nvalid) {
     float* dst = part + (size_t)item * part_stride;
     if (c >= 0 && (p < 0 || p >= a.n_pages)) set_error(a.err, kErrBadPage);
-    if (c < 0 || p < 0 || p >= a.n_pages) {
+    const int n_half = min(32, nvalid - 32 * hf);  // valid keys in this half
+    if (c < 0 || p < 0 || p >= a.n_pages || n_half <= 0) {
       if (lane < G) dst[lane * (D + 2)] = -INFINITY;  // absent
       return;
     }
-    const T* kp = static_cast<const T*>(a.k_pages) + (((size_t)p * a.g + gi) * kChunk) * D;
-    const T* vp = static_cast<const T*>(a.v_pages) + (((size_t)p * a.g + gi) * kChunk) * D;
-    constexpr int CH = D * (int)sizeof(T) / 16;  // 16-byte pieces per row
-    for (int x = lane; x < kChunk * CH; x += 32) {
-      const int r = x / CH, ch = x % CH;
-      const uint32_t bytes = r < nvalid ? 16u : 0u;
-      const size_t src = r < nvalid ? (size_t)r * D + ch * (16 / sizeof(T)) : 0;
-      const uint32_t dk = (uint32_t)__cvta_generic_to_shared(sk + (size_t)r * RS + ch * (16 / sizeof(T)));
-      const uint32_t dv = (uint32_t)__cvta_generic_to_shared(sv + (size_t)r * RS + ch * (16 / sizeof(T)));
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dk), "l"(kp + src), "r"(bytes) : "memory");
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dv), "l"(vp + src), "r"(bytes) : "memory");
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    __syncwarp();
-    const int j0 = lane, j1 = lane + 32;
-    const bool v0 = j0 < nvalid, v1 = j1 < nvalid;
-    float s0[G], s1[G];
+    const size_t row0 = (((size_t)p * a.g + gi) * kChunk + 32 * hf) * D;
+    const T* kp = static_cast<const T*>(a.k_pages) + row0;
+    const T* vp = static_cast<const T*>(a.v_pages) + row0;
+    // Every load of the item is issued up front (its K row for Q.K, lane = key; the
+    // first VB rows of V for P.V, lane = output columns), so the item costs one memory
+    // round trip when VB covers the half.
+    using VRaw = typename RawT<CPL * sizeof(T)>::type;
+    constexpr int VB = CPL * sizeof(T) <= 4 ? 32 : 16;  // V rows per batch (registers)
+    const bool valid = lane < n_half;
+    uint4 kraw[PPR];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) { s0[hh] = 0.f; s1[hh] = 0.f; }
-#pragma unroll 8
-    for (int e = 0; e < D; e += 4) {
-      const float4 k0 = load4(sk + (size_t)j0 * RS + e);
-      const float4 k1 = load4(sk + (size_t)j1 * RS + e);
+    for (int pc = 0; pc < PPR; ++pc)
+      kraw[pc] = valid ? *reinterpret_cast<const uint4*>(kp + (size_t)lane * D + pc * EPP) : make_uint4(0, 0, 0, 0);
+    VRaw vraw[VB];
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float4 qv = *reinterpret_cast<const float4*>(&qS[hh][e]);
-        s0[hh] = fmaf(qv.x, k0.x, fmaf(qv.y, k0.y, fmaf(qv.z, k0.z, fmaf(qv.w, k0.w, s0[hh]))));
-        s1[hh] = fmaf(qv.x, k1.x, fmaf(qv.y, k1.y, fmaf(qv.z, k1.z, fmaf(qv.w, k1.w, s1[hh]))));
+    for (int u = 0; u < VB; ++u)
+      if (u < n_half) vraw[u] = *reinterpret_cast<const VRaw*>(vp + (size_t)u * D + lane * CPL);
+    float s[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) s[hh] = 0.f;
+#pragma unroll
+    for (int pc = 0; pc < PPR; ++pc) {
+      float f[EPP];
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[pc]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 x = __bfloat1622float2(h2[i]);
+          f[2 * i] = x.x;
+          f[2 * i + 1] = x.y;
+        }
+      } else {
+        f[0] = __uint_as_float(kraw[pc].x); f[1] = __uint_as_float(kraw[pc].y);
+        f[2] = __uint_as_float(kraw[pc].z); f[3] = __uint_as_float(kraw[pc].w);
       }
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) s[hh] = fmaf(qS[hh][pc * EPP + e], f[e], s[hh]);
     }
-    float p0[G], p1[G], o[G][CPL];
+    float pr[G], o[G][CPL];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
-      const float a0 = v0 ? s0[hh] * a.scale : -INFINITY;
-      const float a1 = v1 ? s1[hh] * a.scale : -INFINITY;
-      const float m = warp_max(fmaxf(a0, a1));
-      p0[hh] = v0 ? expf(a0 - m) : 0.f;
-      p1[hh] = v1 ? expf(a1 - m) : 0.f;
-      const float l = warp_sum(p0[hh] + p1[hh]);
+      const float x = valid ? s[hh] * a.scale : -INFINITY;
+      const float m = warp_max(x);
+      pr[hh] = valid ? expf(x - m) : 0.f;
+      const float l = warp_sum(pr[hh]);
       if (lane == 0) {
         dst[hh * (D + 2)] = m;
         dst[hh * (D + 2) + 1] = l;
       }
 #pragma unroll
-      for (int x = 0; x < CPL; ++x) o[hh][x] = 0.f;
+      for (int x2 = 0; x2 < CPL; ++x2) o[hh][x2] = 0.f;
     }
-    for (int j = 0; j < nvalid; ++j) {
-      float vj[CPL];
-      if constexpr (CPL == 2) {
-        const float2 f = sizeof(T) == 2
-                             ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sv + (size_t)j * RS + lane * 2))
-                             : *reinterpret_cast<const float2*>(sv + (size_t)j * RS + lane * 2);
-        vj[0] = f.x;
-        vj[1] = f.y;
-      } else {
-        const float4 f = load4(sv + (size_t)j * RS + lane * 4);
-        vj[0] = f.x; vj[1] = f.y; vj[2] = f.z; vj[3] = f.w;
+    // P.V over the rows in registers, then any further batches
+    for (int j0 = 0; j0 < n_half; j0 += VB) {
+      if (j0 > 0) {
+#pragma unroll
+        for (int u = 0; u < VB; ++u)
+          if (j0 + u < n_half) vraw[u] = *reinterpret_cast<const VRaw*>(vp + (size_t)(j0 + u) * D + lane * CPL);
       }
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float pj = __shfl_sync(0xffffffffu, j < 32 ? p0[hh] : p1[hh], j & 31);
+      for (int u = 0; u < VB; ++u) {
+        if (j0 + u >= n_half) break;
+        float vj[CPL];
+        raw_to_f<T, CPL>(vraw[u], vj);
 #pragma unroll
-        for (int x = 0; x < CPL; ++x) o[hh][x] = fmaf(pj, vj[x], o[hh][x]);
+        for (int hh = 0; hh < G; ++hh) {
+          const float pj = __shfl_sync(0xffffffffu, pr[hh], (j0 + u) & 31);
+#pragma unroll
+          for (int x2 = 0; x2 < CPL; ++x2) o[hh][x2] = fmaf(pj, vj[x2], o[hh][x2]);
+        }
       }
     }
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-      for (int x = 0; x < CPL; ++x) dst[hh * (D + 2) + 2 + lane * CPL + x] = o[hh][x];
+      for (int x2 = 0; x2 < CPL; ++x2) dst[hh * (D + 2) + 2 + lane * CPL + x2] = o[hh][x2];
   };
 
   // the own chunk does not depend on the selection: compute it before waiting
   const int own = L > 0 ? (L - 1) / kChunk : 0;
-  if (item == 0 && L > 0)
+  if (item < 2 && L > 0)
     run_item(own, own < a.max_chunks ? a.block_table[(size_t)bi * a.max_chunks + own] : -1, L - own * kChunk);
   pdl_wait_primary();
-  if (item >= 1 && item < n_items && L > 0) {
-    const size_t slot = ((size_t)bi * a.g + gi) * K + item - 1;
+  if (item >= 2 && item < n_items && L > 0) {
+    const size_t slot = ((size_t)bi * a.g + gi) * K + (item >> 1) - 1;
     run_item(a.idx[slot], a.sel_page[slot], kChunk);
   }
 
@@ -472,30 +523,41 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
   if (!s_last) return;
   __threadfence();
   T* out = static_cast<T*>(a.out);
-  // fusion, one warp per head: lane s holds item s (3 rounds cover K + 1 <= 65 items)
+  if (L <= 0) {
+    for (int x = t; x < G * D; x += blockDim.x) out[((size_t)bi * a.h + gi * G) * D + x] = from_f<T>(0.f);
+    if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
+    return;
+  }
+  // fusion weights, one warp per head: lane s handles slot s (3 rounds cover K + 1 <= 65 slots)
   for (int hh = warp; hh < G; hh += kAttWarps) {
-    T* orow = out + ((size_t)bi * a.h + gi * G + hh) * D;
-    if (L <= 0) {
-      for (int x = lane; x < D; x += 32) orow[x] = from_f<T>(0.f);
-      continue;
-    }
     const float* sc_row = a.ssel + ((size_t)bi * a.h + gi * G + hh) * K;
-    float lg[3], mm[3], ll[3];
+    float lg[3], ms[3], ls[3], mh[3][2];
     bool ok[3];
     float M = -INFINITY;
 #pragma unroll
     for (int rr = 0; rr < 3; ++rr) {
-      const int it = lane + 32 * rr;
+      const int sl = lane + 32 * rr;
       ok[rr] = false;
       lg[rr] = -INFINITY;
-      mm[rr] = 0.f;
-      ll[rr] = 1.f;
-      if (it < n_items) {
-        const float* pp = part + (size_t)it * part_stride + hh * (D + 2);
-        mm[rr] = __ldcg(pp);
-        ll[rr] = __ldcg(pp + 1);
-        ok[rr] = mm[rr] != -INFINITY;
-        if (ok[rr]) lg[rr] = it == 0 ? mm[rr] + logf(ll[rr]) : __ldcg(sc_row + it - 1);
+      ms[rr] = -INFINITY;
+      ls[rr] = 0.f;
+      mh[rr][0] = mh[rr][1] = -INFINITY;
+      if (sl < K + 1) {
+        float lh[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float* pp = part + (size_t)(2 * sl + h2) * part_stride + hh * (D + 2);
+          mh[rr][h2] = __ldcg(pp);
+          lh[h2] = mh[rr][h2] != -INFINITY ? __ldcg(pp + 1) : 0.f;
+        }
+        ms[rr] = fmaxf(mh[rr][0], mh[rr][1]);
+        ok[rr] = ms[rr] != -INFINITY;
+        if (ok[rr]) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2)
+            if (mh[rr][h2] != -INFINITY) ls[rr] += lh[h2] * expf(mh[rr][h2] - ms[rr]);
+          lg[rr] = sl == 0 ? ms[rr] + logf(ls[rr]) : __ldcg(sc_row + sl - 1);
+        }
       }
       M = fmaxf(M, lg[rr]);
     }
@@ -506,26 +568,37 @@ __global__ void __launch_bounds__(att_warps<T, D>() * 32) decode_attend_kernel(D
     const float Z = warp_sum(z);
 #pragma unroll
     for (int rr = 0; rr < 3; ++rr) {
-      const int it = lane + 32 * rr;
-      // own: exp(LSE_own - M)/Z * o/l = exp(m - M)/Z * o ; selected: exp(shat - M)/(Z l) * o
-      if (it < n_items)
-        s_w[warp][it] = !ok[rr] ? 0.f : (it == 0 ? expf(mm[rr] - M) / Z : expf(lg[rr] - M) / (Z * ll[rr]));
+      const int sl = lane + 32 * rr;
+      if (sl < K + 1) {
+        // own: exp(LSE_own - M)/Z * o/l = exp(m - M)/Z * o ; selected: exp(shat - M)/(Z l) * o,
+        // with the chunk's (m, l, o) combined from its halves (o_h rescaled by exp(m_h - m))
+        const float wsl = !ok[rr] ? 0.f : (sl == 0 ? expf(ms[rr] - M) / Z : expf(lg[rr] - M) / (Z * ls[rr]));
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+          s_w[hh][2 * sl + h2] = mh[rr][h2] == -INFINITY ? 0.f : wsl * expf(mh[rr][h2] - ms[rr]);
+      }
     }
-    __syncwarp();
-    float acc[CPL];
+  }
+  __syncthreads();
+  // weighted sum of the half-chunk outputs: thread = (head, column); the partials of a
+  // batch of items are all loaded before they are summed
+  constexpr int kFB = 16;
+  for (int x = t; x < G * D; x += blockDim.x) {
+    const int hh = x / D, col = x % D;
+    const float* pc = part + (size_t)hh * (D + 2) + 2 + col;
+    float acc = 0.f;
+    for (int it0 = 0; it0 < n_items; it0 += kFB) {
+      float v[kFB], w[kFB];
 #pragma unroll
-    for (int x = 0; x < CPL; ++x) acc[x] = 0.f;
-#pragma unroll 4
-    for (int it = 0; it < n_items; ++it) {
-      const float w = s_w[warp][it];
-      if (w == 0.f) continue;
-      const float* pp = part + (size_t)it * part_stride + hh * (D + 2) + 2 + lane * CPL;
+      for (int u = 0; u < kFB; ++u) {
+        const int it = it0 + u;
+        w[u] = it < n_items ? s_w[hh][it] : 0.f;
+        v[u] = w[u] != 0.f ? __ldcg(pc + (size_t)it * part_stride) : 0.f;  // absent halves were never written
+      }
 #pragma unroll
-      for (int x = 0; x < CPL; ++x) acc[x] = fmaf(__ldcg(pp + x), w, acc[x]);
+      for (int u = 0; u < kFB; ++u) acc = fmaf(v[u], w[u], acc);
     }
-#pragma unroll
-    for (int x = 0; x < CPL; ++x) orow[lane * CPL + x] = from_f<T>(acc[x]);
-    __syncwarp();
+    out[((size_t)bi * a.h + gi * G + hh) * D + col] = from_f<T>(acc);
   }
   if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
 }
@@ -554,18 +627,11 @@ static cudaError_t launch_decode(DecodeArgs a, cudaStream_t st) {
                              : launch_scan<T, D, G, 8>(a, st);
     if (e != cudaSuccess) return e;
   }
-  constexpr int AW = att_warps<T, D>();
-  constexpr int RS = D + 16 / (int)sizeof(T);
-  constexpr size_t smem = (size_t)AW * 2 * kChunk * RS * sizeof(T);
-  static_assert(smem <= 200 * 1024, "decode attention staging exceeds shared memory");
-  a.att_ctas = (a.top_k + 1 + AW - 1) / AW;
-  cudaError_t e = cudaFuncSetAttribute(decode_attend_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
+  a.att_ctas = (2 * (a.top_k + 1) + kAttWarps - 1) / kAttWarps;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(bg * a.att_ctas);
-  cfg.blockDim = dim3(AW * 32);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(kAttWarps * 32);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

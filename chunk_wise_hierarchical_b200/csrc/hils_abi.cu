@@ -67,7 +67,7 @@ DecodeLayout decode_layout(const hils_shape* s) {
   DecodeLayout L;
   size_t off = kHeader;
   L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
-  L.part_att = off; off = align_up(off + b * g * (K + 1) * G * (d + 2) * 4);
+  L.part_att = off; off = align_up(off + b * g * 2 * (K + 1) * G * (d + 2) * 4);  // half-chunk partials
   L.scan_ticket = off; off = align_up(off + b * g * 4);
   L.att_ticket = off; off = align_up(off + b * g * 4);
   L.idx = off; off = align_up(off + b * g * K * 4);
@@ -336,7 +336,7 @@ StaticLayout static_decode_layout(const hils_shape* s) {
   L.scan_ticket = off; off += kStaticTicketSlots * 4;
   L.att_ticket = off; off += kStaticTicketSlots * 4;
   L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
-  L.part_att = off; off = align_up(off + b * g * (K + 1) * G * (d + 2) * 4);
+  L.part_att = off; off = align_up(off + b * g * 2 * (K + 1) * G * (d + 2) * 4);  // half-chunk partials
   L.idx = off; off = align_up(off + b * g * K * 4);
   L.sel_page = off; off = align_up(off + b * g * K * 4);
   L.ssel = off; off = align_up(off + b * h * K * 4);

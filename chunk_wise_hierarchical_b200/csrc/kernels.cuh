@@ -53,7 +53,7 @@ struct DecodeArgs {
   int32_t* sel_page;           // [b,g,K] page of each selected chunk
   float* ssel;                 // [b,h,K]
   unsigned long long* part_keys;  // [b,g,nsplit,K] per-range Top-K lists
-  float* part_att;             // [b,g,K+1,G,d+2]
+  float* part_att;             // [b,g,2(K+1),G,d+2]: per half chunk (max, sum, unnormalised output)
   unsigned* scan_ticket;       // [b,g] (the scan uses entry (b, 0))
   unsigned* att_ticket;        // [b,g]
   unsigned* err;
