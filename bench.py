@@ -57,6 +57,28 @@ def decode_bytes(cfg):
     return float(kv + summ + qo), float(kv)
 
 
+# DRAM bytes (read + write) per launch of the prefill attention kernel at the bench size,
+# from one ncu capture (`ncu --set full --clock-control none -k regex:attend_tc_kernel -s 3
+# -c 1 python bench.py --steps 3 --warmup 3 --no-decode --no-cpu`, summarised under
+# profiles/).  Reported only while the kernel's sources are the ones it was taken on.
+ATTEND_TRAFFIC = {
+    "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc.cu":
+                "c8500ff5a6374bea5ab48e689ed9ce21b7a8493011b381219bf932f260a03478",
+                "chunk_wise_hierarchical_b200/csrc/tc_util.cuh":
+                "2c8199fc4ff66b314758faa3af3800696b99b5856f4f2dcdf03a90bd6e6727b6"},
+    "bytes": 269144832 + 54669824,
+}
+
+
+def attend_traffic():
+    import hashlib
+    for rel, digest in ATTEND_TRAFFIC["sources"].items():
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    return ATTEND_TRAFFIC["bytes"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -375,7 +397,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": "attend_selected (selected + own chunk attention, fusion)",
                      "achieved": round(att_tflops, 3), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": round(att_tflops / bf16_peak, 5), "peak_source": f"{peak_src} bf16 burst",
-                     "traffic": args.traffic},
+                     "traffic": args.traffic if args.traffic is not None else attend_traffic()},
         "e2e": {"value": round(job_tflops(ws_world, flops, pre["ms_e2e"]), 4), "unit": "TFLOP/s",
                 "ms_per_step": round(pre["ms_e2e"], 3), "h2d_bytes_per_step": pre["h2d"],
                 "d2h_bytes_per_step": pre["d2h"]},
