@@ -45,14 +45,14 @@ def algorithmic_flops(batch, heads_q, seq_len, head_dim, top_k, chunk=64):
     return float(4 * head_dim * keys.sum() * batch * heads_q)
 
 
-def decode_bytes(cfg):
+def decode_bytes(cfg, summary_bytes=4):
     b, h, g, d, K = cfg["batch"], cfg["heads_q"], cfg["heads_kv"], cfg["head_dim"], cfg["top_k"]
     L = cfg["seq_len"]
     own = (L - 1) // 64
     keff = min(K, own)
     own_keys = L - own * 64
     kv = b * g * (keff * 64 + own_keys) * d * 2 * 2
-    summ = b * own * h * (d + 1) * 4
+    summ = b * own * h * (d * summary_bytes + 4)  # kbar (fp32 or bf16 cache) + fp32 H
     qo = b * h * d * 2 * 2
     return float(kv + summ + qo), float(kv)
 
@@ -302,6 +302,8 @@ def run_prefill(args, ws_world, rank, local):
 
 # ---------------------------------------------------------------------------- decode (ours)
 def run_decode(name, n_caches, dev, reps=50):
+    """Decode step time for the fp32 summary cache and for the compact bf16 one, on the
+    same inputs: CUDA-graph replays rotating over n_caches independent caches."""
     import chunk_wise_hierarchical_b200 as hils
     cfg = CONFIGS[name]
     K = cfg["top_k"]
@@ -310,43 +312,50 @@ def run_decode(name, n_caches, dev, reps=50):
         di = decode_inputs(seed=100 + c, device=dev, **cfg)
         P, g, B, d = di.k_pages.shape
         h = di.landmark_pages.shape[1]
-        kbar = torch.empty((P, h, d), dtype=torch.float32, device=dev)
-        hb = torch.empty((P, h), dtype=torch.float32, device=dev)
-        hils.summarize_paged(di.k_pages, di.landmark_pages, torch.arange(P, dtype=torch.int32, device=dev),
-                             kbar, hb)
+        ids = torch.arange(P, dtype=torch.int32, device=dev)
+        kbars = {}
+        for dt in (torch.float32, torch.bfloat16):
+            kbar = torch.empty((P, h, d), dtype=dt, device=dev)
+            hb = torch.empty((P, h), dtype=torch.float32, device=dev)
+            hils.summarize_paged(di.k_pages, di.landmark_pages, ids, kbar, hb)
+            kbars[dt] = (kbar, hb)
         call = hils.Decode(cfg["batch"], h, g, d, di.max_chunks, K, torch.bfloat16, device=dev)
         out = torch.empty_like(di.q)
         del di.landmark_pages
-        caches.append((di, kbar, hb, call, out))
+        caches.append((di, kbars, call, out))
     torch.cuda.synchronize()
     s = torch.cuda.Stream(device=dev)
-    graphs = []
-    with torch.cuda.stream(s):
-        for (di, kbar, hb, call, out) in caches:  # warm up outside capture
-            call(di.q, di.k_pages, di.v_pages, kbar, hb, di.block_table, di.seq_lens, out=out)
-    torch.cuda.synchronize()
-    for (di, kbar, hb, call, out) in caches:
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=s):
-            call(di.q, di.k_pages, di.v_pages, kbar, hb, di.block_table, di.seq_lens, out=out)
-        graphs.append(gr)
-    for gr in graphs:
-        gr.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for r in range(reps):
-        graphs[r % len(graphs)].replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
-    for (di, kbar, hb, call, out) in caches:
-        assert call.device_status() == 0
-    alg, kv_only = decode_bytes(cfg)
-    del graphs, caches
+    res = {}
+    for dt, sbytes in ((torch.float32, 4), (torch.bfloat16, 2)):
+        graphs = []
+        with torch.cuda.stream(s):
+            for (di, kbars, call, out) in caches:  # warm up outside capture
+                call(di.q, di.k_pages, di.v_pages, *kbars[dt], di.block_table, di.seq_lens, out=out)
+        torch.cuda.synchronize()
+        for (di, kbars, call, out) in caches:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=s):
+                call(di.q, di.k_pages, di.v_pages, *kbars[dt], di.block_table, di.seq_lens, out=out)
+            graphs.append(gr)
+        for gr in graphs:
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for r in range(reps):
+            graphs[r % len(graphs)].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        for (di, kbars, call, out) in caches:
+            assert call.device_status() == 0
+        alg, kv_only = decode_bytes(cfg, sbytes)
+        del graphs
+        res[dt] = dict(ms=ms, tok_s=cfg["batch"] / (ms * 1e-3), gbs=alg / (ms * 1e-3) / 1e9, bytes=alg,
+                       kv_bytes=kv_only)
+    del caches
     torch.cuda.empty_cache()
-    return dict(ms=ms, tok_s=cfg["batch"] / (ms * 1e-3), gbs=alg / (ms * 1e-3) / 1e9, bytes=alg,
-                kv_bytes=kv_only)
+    return res
 
 
 def run_ours(args):
@@ -357,7 +366,9 @@ def run_ours(args):
     if not args.no_decode:
         for name in args.decode_configs.split(","):
             nc = 3 if name == "decode_32k" else 1   # 3 rotating caches keep 32K out of L2
-            dec[name] = run_decode(name, nc, torch.device("cuda", local))
+            r = run_decode(name, nc, torch.device("cuda", local))
+            dec[name] = r[torch.float32]
+            dec[name + "_bf16_summaries"] = r[torch.bfloat16]
     if args.decode_only:
         if rank == 0:
             print(json.dumps({"decode": {k: {"us_per_step": round(r["ms"] * 1e3, 2),

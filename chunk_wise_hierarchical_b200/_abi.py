@@ -65,6 +65,8 @@ def lib():
         "hils_attend": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "hils_attend_selected": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "hils_decode": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
+        "hils_summarize_paged_ex": (i32, [S, _P, _P, _P, i32, i32, _P, i32, _P, _P]),
+        "hils_decode_ex": (i32, [S, _P, _P, _P, _P, i32, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
         "hils_decode_static": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, _P]),
         "hils_device_status": (i32, [_P, _P]),
     }
@@ -77,7 +79,7 @@ def lib():
 
 
 EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_decode",
-            "hils_decode_static", "hils_device_status", "hils_select", "hils_status_string", "hils_summarize",
+            "hils_decode_ex", "hils_decode_static", "hils_device_status", "hils_summarize_paged_ex", "hils_select", "hils_status_string", "hils_summarize",
             "hils_summarize_paged", "hils_workspace_size"]
 
 
@@ -141,15 +143,16 @@ def summarize(k, landmark, scale=None, stream=None):
 
 
 def summarize_paged(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages, scale=None, stream=None):
-    """Writes the summaries of the listed pages into kbar_pages / hbias_pages."""
+    """Writes the summaries of the listed pages into kbar_pages (fp32, or bf16 for the
+    compact cache) / hbias_pages (fp32)."""
     n_pages, g, chunk, d = k_pages.shape
     h = landmark_pages.shape[1]
     if page_ids.dtype != torch.int32:
         raise TypeError("page_ids must be int32")
     sh = make_shape(0, h, g, d, 0, 0, _dt(k_pages), chunk=chunk, scale=scale or 0.0)
-    _check(lib().hils_summarize_paged(ctypes.byref(sh), _ptr(k_pages), _ptr(landmark_pages), _ptr(page_ids),
-                                      int(page_ids.numel()), int(n_pages), _ptr(kbar_pages),
-                                      _ptr(hbias_pages), _stream(stream)), "hils_summarize_paged")
+    _check(lib().hils_summarize_paged_ex(ctypes.byref(sh), _ptr(k_pages), _ptr(landmark_pages), _ptr(page_ids),
+                                         int(page_ids.numel()), int(n_pages), _ptr(kbar_pages), _dt(kbar_pages),
+                                         _ptr(hbias_pages), _stream(stream)), "hils_summarize_paged_ex")
 
 
 def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True):
@@ -191,10 +194,20 @@ class Prefill:
         return lib().hils_device_status(_ptr(self.ws), _stream(stream))
 
 
-def attend(q, k, v, landmark, top_k, scale=None, stream=None, return_idx=False):
-    """HiLS prefill forward; returns out (and topk_idx if asked)."""
+def attend(q, k, v, landmark, top_k, scale=None, stream=None, return_idx=False, q_score=None):
+    """HiLS prefill forward; returns out (and topk_idx if asked).
+
+    q_score: a separate scoring query (the Q-Cal interface): summaries, then
+    hils_select with q_score, then hils_attend_selected with q."""
     b, h, n, d = q.shape
     g = k.shape[1]
+    if q_score is not None:
+        if q_score.shape != q.shape or q_score.dtype != q.dtype:
+            raise ValueError("q_score must match q's shape and dtype")
+        kbar, hb = summarize(k, landmark, scale=scale, stream=stream)
+        idx, sc = select(q_score, kbar, hb, top_k, g, scale=scale, stream=stream)
+        out = attend_selected(q, k, v, idx, sc, scale=scale, stream=stream)
+        return (out, idx) if return_idx else out
     call = Prefill(b, h, g, n, d, top_k, q.dtype, scale=scale, device=q.device)
     idx = torch.empty((b, g, n, top_k), dtype=torch.int32, device=q.device) if return_idx else None
     out = call(q, k, v, landmark, topk_idx=idx, stream=stream)
@@ -239,10 +252,10 @@ class Decode:
             raise ValueError("block_table must be [batch, max_chunks]")
         if out is None:
             out = torch.empty_like(q)
-        _check(lib().hils_decode(ctypes.byref(s), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kbar_pages),
-                                 _ptr(hbias_pages), _ptr(block_table), self.max_chunks, _ptr(seq_lens),
-                                 int(k_pages.shape[0]), _ptr(out), _ptr(topk_idx), _ptr(self.ws),
-                                 self.ws.numel(), _stream(stream)), "hils_decode")
+        _check(lib().hils_decode_ex(ctypes.byref(s), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kbar_pages),
+                                    _dt(kbar_pages), _ptr(hbias_pages), _ptr(block_table), self.max_chunks,
+                                    _ptr(seq_lens), int(k_pages.shape[0]), _ptr(out), _ptr(topk_idx), _ptr(self.ws),
+                                    self.ws.numel(), _stream(stream)), "hils_decode_ex")
         return out
 
     def device_status(self, stream=None):

@@ -130,13 +130,18 @@ __device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, 
 // (atomic ticket; no CTA waits on another) merges the ranges' lists.
 // Four CTAs per SM (64 registers a thread): a page gather's bandwidth grows with the
 // warps resident on the SM far more than with the loads each warp has in flight.
-template <typename T, int D, int G, int FPT>
+// S: element type of the cached summaries (fp32, or bf16 for the compact cache).
+// MULTI: a page's block is narrower than the CTA, so one load step covers several pages.
+template <typename T, int D, int G, typename S, int FPT, bool MULTI>
 __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) float s_score[];  // [range][h]; reused by the merge
   __shared__ int s_page[kMaxRange];
   __shared__ int s_last;
-  constexpr int QPR = D / 4;                     // float4 per head row
-  constexpr int PB = FPT >= 8 ? 1 : 8 / FPT;     // pages per batch of loads
+  constexpr int EPP = 16 / (int)sizeof(S);       // summary elements per 16-byte piece
+  constexpr int QPR = D / EPP;                   // pieces per head row
+  // load steps per batch: 8 pages' worth of fp32 pieces per thread (bf16 pieces hold twice
+  // the elements, so half the steps keep the registers the same)
+  constexpr int PB = FPT >= 8 ? 1 : (8 / FPT) * 4 / EPP > 0 ? (8 / FPT) * 4 / EPP : 1;
 
   pdl_launch_dependents();  // the attend grid may start its selection-independent prologue
   const int t = threadIdx.x, warp = t >> 5;
@@ -150,34 +155,42 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
   const int n_cand = min(own, a.max_chunks);
   const int nc = max(0, min(n_cand, c_lo + R) - c_lo);
   for (int x = t; x < nc; x += kScanThreads) s_page[x] = bt[c_lo + x];
-  const int F = H * QPR;  // float4 per page block
-  float4 qv[FPT];
+  // A page's summaries [h][d] are F 16-byte pieces.  When a page block is smaller than
+  // the CTA, one load step covers PPI pages (thread t: page t / F, piece t % F);
+  // otherwise thread t takes pieces t + 256 k of one page.
+  const int F = H * QPR;
+  const int PPI = MULTI ? kScanThreads / F : 1;
+  const int w = MULTI ? t / F : 0;
+  const int fl = MULTI ? t % F : t;
+  const bool tw = !MULTI || w < PPI;
+  float qf[FPT][EPP];
 #pragma unroll
   for (int k = 0; k < FPT; ++k) {
-    const int f = t + k * kScanThreads;
-    qv[k] = f < F ? load4(static_cast<const T*>(a.q) + ((size_t)bi * H + f / QPR) * D + (f % QPR) * 4)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int f = fl + k * kScanThreads;
+    const T* qp = static_cast<const T*>(a.q) + ((size_t)bi * H + f / QPR) * D + (f % QPR) * EPP;
+#pragma unroll
+    for (int e = 0; e < EPP; ++e) qf[k][e] = tw && f < F ? to_f(qp[e]) : 0.f;
   }
   __syncthreads();
 
-  // Pages are processed in batches of PB: the batch's loads are all in flight before
-  // the first is reduced.
-  const float4* kb4 = reinterpret_cast<const float4*>(a.kbar_pages);
+  // Pages are processed in batches of PB load steps: the batch's loads are all in flight
+  // before the first is reduced.
+  const uint4* kb16 = reinterpret_cast<const uint4*>(a.kbar_pages);
   struct Batch {
-    float4 kv[PB][FPT];
+    uint4 kv[PB][FPT];
     float hv[PB][FPT];  // H of the lane's head (read by the lane that writes the score)
     int pg[PB];
   };
   auto load = [&](Batch& B, int j0) {
 #pragma unroll
     for (int u = 0; u < PB; ++u) {
-      const int j = j0 + u;
-      B.pg[u] = j < nc ? s_page[j] : -1;
+      const int j = j0 + u * PPI + w;
+      B.pg[u] = tw && j < nc ? s_page[j] : -1;
       const bool ok = B.pg[u] >= 0 && B.pg[u] < a.n_pages;
 #pragma unroll
       for (int k = 0; k < FPT; ++k) {
-        const int f = t + k * kScanThreads;
-        B.kv[u][k] = ok && f < F ? __ldg(kb4 + (size_t)B.pg[u] * F + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int f = fl + k * kScanThreads;
+        B.kv[u][k] = ok && f < F ? __ldg(kb16 + (size_t)B.pg[u] * F + f) : make_uint4(0, 0, 0, 0);
         B.hv[u][k] = ok && f < F && f % QPR == 0 ? __ldg(a.hbias_pages + (size_t)B.pg[u] * H + f / QPR) : 0.f;
       }
     }
@@ -185,15 +198,29 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
   auto reduce = [&](const Batch& B, int j0) {
 #pragma unroll
     for (int u = 0; u < PB; ++u) {
-      const int j = j0 + u;
+      const int j = j0 + u * PPI + w;
 #pragma unroll
       for (int k = 0; k < FPT; ++k) {
-        const int f = t + k * kScanThreads;
-        const float4 kv = B.kv[u][k];
-        float dot = fmaf(qv[k].x, kv.x, fmaf(qv[k].y, kv.y, fmaf(qv[k].z, kv.z, qv[k].w * kv.w)));
+        const int f = fl + k * kScanThreads;
+        float x[EPP];
+        if constexpr (sizeof(S) == 2) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&B.kv[u][k]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 y = __bfloat1622float2(h2[i]);
+            x[2 * i] = y.x;
+            x[2 * i + 1] = y.y;
+          }
+        } else {
+          x[0] = __uint_as_float(B.kv[u][k].x); x[1] = __uint_as_float(B.kv[u][k].y);
+          x[2] = __uint_as_float(B.kv[u][k].z); x[3] = __uint_as_float(B.kv[u][k].w);
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) dot = fmaf(qf[k][e], x[e], dot);
 #pragma unroll
         for (int o = QPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        if (j < nc && f < F && f % QPR == 0) {
+        if (tw && j < nc && f < F && f % QPR == 0) {
           const int head = f / QPR, p = B.pg[u];
           float sc = NAN;
           if (p >= 0 && p < a.n_pages) sc = fmaf(dot, a.scale, B.hv[u][k]);
@@ -203,7 +230,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       }
     }
   };
-  for (int j0 = 0; j0 < nc; j0 += PB) {
+  for (int j0 = 0; j0 < nc; j0 += PB * PPI) {
     Batch bt_;
     load(bt_, j0);
     reduce(bt_, j0);
@@ -330,11 +357,11 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       float sc = -INFINITY;
       if (c >= 0) {
         const int p = bt[c];
-        const float* kb = a.kbar_pages + ((size_t)p * H + gi * G + hh) * D;
+        const S* kb = static_cast<const S*>(a.kbar_pages) + ((size_t)p * H + gi * G + hh) * D;
         const T* qr = static_cast<const T*>(a.q) + ((size_t)bi * H + gi * G + hh) * D;
         float acc = 0.f;
 #pragma unroll
-        for (int e = lane; e < D; e += 32) acc = fmaf(to_f(qr[e]), __ldg(kb + e), acc);
+        for (int e = lane; e < D; e += 32) acc = fmaf(to_f(qr[e]), to_f(kb[e]), acc);
         acc = warp_sum(acc);
         sc = fmaf(acc, a.scale, __ldg(a.hbias_pages + (size_t)p * H + gi * G + hh));
       }
@@ -603,14 +630,25 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
   if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
 }
 
-template <typename T, int D, int G, int FPT>
+template <typename T, int D, int G, typename S, int FPT, bool MULTI = false>
 static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores
-  cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, FPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, S, FPT, MULTI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_scan_kernel<T, D, G, FPT><<<(unsigned)a.b * a.nsplit, kScanThreads, smem, st>>>(a);
+  decode_scan_kernel<T, D, G, S, FPT, MULTI><<<(unsigned)a.b * a.nsplit, kScanThreads, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+template <typename T, int D, int G, typename S>
+static cudaError_t launch_scan_by_width(const DecodeArgs& a, cudaStream_t st) {
+  const int f16 = a.h * D * (int)sizeof(S) / 16;  // 16-byte pieces per page of summaries
+  const int fpt = (f16 + kScanThreads - 1) / kScanThreads;
+  if (f16 < kScanThreads) return launch_scan<T, D, G, S, 1, true>(a, st);
+  return fpt <= 1 ? launch_scan<T, D, G, S, 1>(a, st)
+       : fpt <= 2 ? launch_scan<T, D, G, S, 2>(a, st)
+       : fpt <= 4 ? launch_scan<T, D, G, S, 4>(a, st)
+                  : launch_scan<T, D, G, S, 8>(a, st);
 }
 
 template <typename T, int D, int G>
@@ -619,12 +657,13 @@ static cudaError_t launch_decode(DecodeArgs a, cudaStream_t st) {
   if (bg == 0) return cudaSuccess;
   if (!decode_supported(a.h, D)) return cudaErrorInvalidValue;
   if (a.top_k > 0) {
-    const int f4 = a.h * D / 4;  // float4 per page of summaries
-    const int fpt = (f4 + kScanThreads - 1) / kScanThreads;
-    cudaError_t e = fpt <= 1 ? launch_scan<T, D, G, 1>(a, st)
-                  : fpt <= 2 ? launch_scan<T, D, G, 2>(a, st)
-                  : fpt <= 4 ? launch_scan<T, D, G, 4>(a, st)
-                             : launch_scan<T, D, G, 8>(a, st);
+    cudaError_t e;
+    if (a.kbar_bf16) {
+      if constexpr (sizeof(T) == 2) e = launch_scan_by_width<T, D, G, __nv_bfloat16>(a, st);
+      else return cudaErrorInvalidValue;  // the compact summary cache is for bf16 models
+    } else {
+      e = launch_scan_by_width<T, D, G, float>(a, st);
+    }
     if (e != cudaSuccess) return e;
   }
   a.att_ctas = (2 * (a.top_k + 1) + kAttWarps - 1) / kAttWarps;

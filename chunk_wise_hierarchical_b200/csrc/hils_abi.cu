@@ -156,8 +156,17 @@ hils_status hils_summarize(const hils_shape* s, const void* k, const void* landm
 hils_status hils_summarize_paged(const hils_shape* s, const void* k_pages, const void* landmark_pages,
                                  const int32_t* page_ids, int32_t n_listed, int32_t n_pages,
                                  float* kbar_pages, float* hbias_pages, void* stream) {
+  return hils_summarize_paged_ex(s, k_pages, landmark_pages, page_ids, n_listed, n_pages, kbar_pages, HILS_F32,
+                                 hbias_pages, stream);
+}
+
+hils_status hils_summarize_paged_ex(const hils_shape* s, const void* k_pages, const void* landmark_pages,
+                                    const int32_t* page_ids, int32_t n_listed, int32_t n_pages,
+                                    void* kbar_pages, int32_t summary_dtype, float* hbias_pages, void* stream) {
   hils_status st = check_shape(s, false);
   if (st != HILS_OK) return st;
+  if (summary_dtype != HILS_F32 && summary_dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+  if (summary_dtype == HILS_BF16 && s->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
   if (n_listed < 0 || n_pages < 0) return HILS_ERR_INVALID_ARG;
   if (n_listed == 0) return HILS_OK;
   if (!k_pages || !landmark_pages || !page_ids || !kbar_pages || !hbias_pages) return HILS_ERR_INVALID_ARG;
@@ -167,6 +176,7 @@ hils_status hils_summarize_paged(const hils_shape* s, const void* k_pages, const
   a.b = 0; a.h = s->heads_q; a.g = s->heads_kv; a.n = 0; a.d = s->head_dim; a.n_chunks = 0;
   a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
   a.page_ids = page_ids; a.n_listed = n_listed; a.n_pages = n_pages;
+  a.kbar_bf16 = summary_dtype == HILS_BF16;
   return cuda_status(hils::run_summarize(a, (cudaStream_t)stream));
 }
 
@@ -250,8 +260,19 @@ hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages,
                         const float* kbar_pages, const float* hbias_pages, const int32_t* block_table,
                         int32_t max_chunks, const int32_t* seq_lens, int32_t n_pages, void* out,
                         int32_t* topk_idx_out, void* ws, size_t ws_bytes, void* stream) {
+  return hils_decode_ex(s, q, k_pages, v_pages, kbar_pages, HILS_F32, hbias_pages, block_table, max_chunks,
+                        seq_lens, n_pages, out, topk_idx_out, ws, ws_bytes, stream);
+}
+
+hils_status hils_decode_ex(const hils_shape* s, const void* q, const void* k_pages, const void* v_pages,
+                           const void* kbar_pages, int32_t summary_dtype, const float* hbias_pages,
+                           const int32_t* block_table, int32_t max_chunks, const int32_t* seq_lens,
+                           int32_t n_pages, void* out, int32_t* topk_idx_out, void* ws, size_t ws_bytes,
+                           void* stream) {
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
+  if (summary_dtype != HILS_F32 && summary_dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+  if (summary_dtype == HILS_BF16 && s->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
   if (s->batch == 0) return HILS_OK;
   if (!hils::decode_supported(s->heads_q, s->head_dim)) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
@@ -281,6 +302,7 @@ hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages,
   da.b = s->batch; da.h = s->heads_q; da.g = s->heads_kv; da.d = s->head_dim; da.top_k = s->top_k;
   da.max_chunks = max_chunks; da.n_pages = n_pages; da.scale = eff_scale(s);
   da.bf16 = s->dtype == HILS_BF16;
+  da.kbar_bf16 = summary_dtype == HILS_BF16;
   return cuda_status(hils::run_decode(da, cs));
 }
 

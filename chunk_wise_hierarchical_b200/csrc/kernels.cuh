@@ -12,12 +12,13 @@ namespace hils {
 struct SummarizeArgs {
   const void* k;          // [b,g,N,d] or pages [P,g,B,d]
   const void* lm;         // [b,h,C,d] or pages [P,h,d]
-  float* kbar;            // [b,h,C,d] or [P,h,d]
+  void* kbar;             // [b,h,C,d] or [P,h,d]: fp32, or bf16 when kbar_bf16 (paged only)
   float* hbias;           // [b,h,C]   or [P,h]
   int b, h, g, n, d, n_chunks;
   float scale;
   bool bf16;
   const int32_t* page_ids;  // nullptr: contiguous mode
+  bool kbar_bf16;
   int n_listed, n_pages;
 };
 cudaError_t run_summarize(const SummarizeArgs& a, cudaStream_t st);
@@ -44,7 +45,7 @@ struct DecodeArgs {
   const void* q;               // [b,h,d]
   const void* k_pages;         // [P,g,B,d]
   const void* v_pages;
-  const float* kbar_pages;     // [P,h,d]
+  const void* kbar_pages;      // [P,h,d] fp32, or bf16 when kbar_bf16
   const float* hbias_pages;    // [P,h]
   const int32_t* block_table;  // [b,max_chunks]
   const int32_t* seq_lens;     // [b]
@@ -57,6 +58,7 @@ struct DecodeArgs {
   unsigned* scan_ticket;       // [b,g] (the scan uses entry (b, 0))
   unsigned* att_ticket;        // [b,g]
   unsigned* err;
+  bool kbar_bf16;              // compact summary cache (bf16 models only)
   int b, h, g, d, top_k, max_chunks, n_pages;
   int nsplit, range, att_ctas; // set by the launcher: scan ranges per sequence, chunks per range
   float scale;

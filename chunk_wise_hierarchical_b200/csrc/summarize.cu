@@ -11,9 +11,10 @@
 
 namespace hils {
 
-template <typename T, int D>
+// KB: element type of the written kbar (fp32, or bf16 for a compact paged summary cache).
+template <typename T, int D, typename KB>
 __global__ void __launch_bounds__(128) summarize_kernel(
-    const T* __restrict__ k, const T* __restrict__ lm, float* __restrict__ kbar,
+    const T* __restrict__ k, const T* __restrict__ lm, KB* __restrict__ kbar,
     float* __restrict__ hbias, int h, int g, int n_seq, int n_chunks, float scale,
     const int32_t* __restrict__ page_ids, int n_pages) {
   __shared__ float kS[kChunk][D + 1];
@@ -26,7 +27,7 @@ __global__ void __launch_bounds__(128) summarize_kernel(
   const T* kbase;
   const T* lbase;      // landmark of query head (gi * grp) for this chunk
   size_t lm_head_stride, out_head_stride, hb_head_stride;
-  float* kb_out;
+  KB* kb_out;
   float* hb_out;
   if (page_ids == nullptr) {
     // blockIdx.x = ((bi * g) + gi) * n_chunks + c
@@ -95,21 +96,25 @@ __global__ void __launch_bounds__(128) summarize_kernel(
       float acc = 0.f;
 #pragma unroll 8
       for (int j = 0; j < kChunk; ++j) acc = fmaf(pS[j], kS[j][e], acc);
-      kb_out[hh * out_head_stride + e] = acc;
+      kb_out[hh * out_head_stride + e] = from_f<KB>(acc);
     }
     if (tid == 0) hb_out[hh * hb_head_stride] = logf(z) - zs / z;
   }
 }
 
 template <typename T, int D>
-static cudaError_t launch_summarize(const T* k, const T* lm, float* kbar, float* hbias, int b, int h,
-                                    int g, int n_seq, int n_chunks, float scale,
+static cudaError_t launch_summarize(const T* k, const T* lm, void* kbar, bool kbar_bf16, float* hbias, int b,
+                                    int h, int g, int n_seq, int n_chunks, float scale,
                                     const int32_t* page_ids, int n_listed, int n_pages,
                                     cudaStream_t st) {
   unsigned blocks = page_ids ? (unsigned)n_listed * g : (unsigned)b * g * n_chunks;
   if (blocks == 0) return cudaSuccess;
-  summarize_kernel<T, D><<<blocks, 128, 0, st>>>(k, lm, kbar, hbias, h, g, n_seq, n_chunks, scale,
-                                                  page_ids, n_pages);
+  if (kbar_bf16)
+    summarize_kernel<T, D, __nv_bfloat16><<<blocks, 128, 0, st>>>(
+        k, lm, static_cast<__nv_bfloat16*>(kbar), hbias, h, g, n_seq, n_chunks, scale, page_ids, n_pages);
+  else
+    summarize_kernel<T, D, float><<<blocks, 128, 0, st>>>(k, lm, static_cast<float*>(kbar), hbias, h, g, n_seq,
+                                                          n_chunks, scale, page_ids, n_pages);
   return cudaGetLastError();
 }
 
@@ -118,17 +123,17 @@ cudaError_t run_summarize(const SummarizeArgs& a, cudaStream_t st) {
     auto k = static_cast<const __nv_bfloat16*>(a.k);
     auto l = static_cast<const __nv_bfloat16*>(a.lm);
     if (a.d == 64)
-      return launch_summarize<__nv_bfloat16, 64>(k, l, a.kbar, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks,
+      return launch_summarize<__nv_bfloat16, 64>(k, l, a.kbar, a.kbar_bf16, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks,
                                                  a.scale, a.page_ids, a.n_listed, a.n_pages, st);
-    return launch_summarize<__nv_bfloat16, 128>(k, l, a.kbar, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks,
+    return launch_summarize<__nv_bfloat16, 128>(k, l, a.kbar, a.kbar_bf16, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks,
                                                 a.scale, a.page_ids, a.n_listed, a.n_pages, st);
   }
   auto k = static_cast<const float*>(a.k);
   auto l = static_cast<const float*>(a.lm);
   if (a.d == 64)
-    return launch_summarize<float, 64>(k, l, a.kbar, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks, a.scale,
+    return launch_summarize<float, 64>(k, l, a.kbar, a.kbar_bf16, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks, a.scale,
                                        a.page_ids, a.n_listed, a.n_pages, st);
-  return launch_summarize<float, 128>(k, l, a.kbar, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks, a.scale,
+  return launch_summarize<float, 128>(k, l, a.kbar, a.kbar_bf16, a.hbias, a.b, a.h, a.g, a.n, a.n_chunks, a.scale,
                                       a.page_ids, a.n_listed, a.n_pages, st);
 }
 

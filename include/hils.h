@@ -252,6 +252,31 @@ HILS_API hils_status hils_decode_static(const hils_shape* shape, const void* q, 
                         void* stream);
 
 /*
+ * hils_summarize_paged_ex, hils_decode_ex -- hils_summarize_paged and
+ * hils_decode with the cached summaries kbar_pages stored in summary_dtype:
+ * HILS_F32 (the plain entry points) or HILS_BF16, a compact cache that
+ * halves the bytes the decode scan reads (the summaries of a 512K context
+ * are most of a decode step's memory traffic).  Scores from bf16 summaries
+ * carry the bf16 rounding of kbar (relative error up to 2^-9 per element,
+ * about 2^-9 |q||kbar| * scale on a score), so their Top-K may differ from
+ * the fp32 cache's where candidate keys lie that close.  H stays fp32.
+ * HILS_BF16 summaries require shape.dtype == HILS_BF16 (HILS_ERR_UNSUPPORTED
+ * otherwise); an unknown summary_dtype is HILS_ERR_INVALID_ARG.  The HiLS
+ * pages fix no storage precision for kbar; the bf16 cache is an option of
+ * this library.
+ */
+HILS_API hils_status hils_summarize_paged_ex(const hils_shape* shape, const void* k_pages,
+                                    const void* landmark_pages, const int32_t* page_ids,
+                                    int32_t n_listed, int32_t n_pages, void* kbar_pages,
+                                    int32_t summary_dtype, float* hbias_pages, void* stream);
+HILS_API hils_status hils_decode_ex(const hils_shape* shape, const void* q, const void* k_pages,
+                           const void* v_pages, const void* kbar_pages, int32_t summary_dtype,
+                           const float* hbias_pages, const int32_t* block_table,
+                           int32_t max_chunks, const int32_t* seq_lens, int32_t n_pages,
+                           void* out, int32_t* topk_idx_out, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
  * hils_device_status -- synchronises `stream`, reads and clears the error
  * word at the start of a hils_attend / hils_attend_selected / hils_decode
  * workspace, and returns HILS_OK, HILS_ERR_DEVICE_CHECK or

@@ -196,14 +196,17 @@ def _softmax_attend(qv, keys, vals, sc):
 
 
 def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
-            forced_idx=None, rows=None, heads=None):
+            forced_idx=None, rows=None, heads=None, q_score=None):
     """HiLS forward for a contiguous causal sequence.
 
     q [b,h,N,d], k/v [b,g,N,d], landmark [b,h,C,d] (C = N // chunk).
     mode: "landmark" or "exact".  forced_idx [b,g,R,K]: selection supplied by
     the caller (-1 = unused slot).  rows: query positions (default all);
     heads: (b, h) pairs to produce (default all; selection still uses the
-    whole GQA group).
+    whole GQA group).  q_score [b,h,N,d]: a separate scoring query (notes
+    section 5.4, the Q-Cal interface): it replaces q in the chunk scores, so it
+    decides the selection and the inter-chunk weights, while q keeps the
+    intra-chunk attention and the own chunk.
 
     Returns a dict with out [b,h,R,d] (nan for heads not produced),
     idx [b,g,R,K], shat_sel [b,h,R,K] (-inf in unused slots), lse_own
@@ -215,11 +218,12 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
     grp = h // g
     sc = _scale(d, scale)
     rows = np.arange(n) if rows is None else np.asarray(rows)
+    qs64 = q64 if q_score is None else _f64(q_score)
     if mode == "landmark":
         kbar, hb = summarize(k64, landmark, chunk, scale)
-        shat = chunk_scores(q64, kbar, hb, chunk, scale, rows)
+        shat = chunk_scores(qs64, kbar, hb, chunk, scale, rows)
     elif mode == "exact":
-        shat = exact_chunk_lse(q64, k64, chunk, scale, rows)
+        shat = exact_chunk_lse(qs64, k64, chunk, scale, rows)
     else:
         raise ValueError(mode)
     if forced_idx is None:

@@ -118,6 +118,29 @@ def test_select_one_head_per_group_bf16(kw):
     assert np.array_equal((gi >= 0).sum(-1), np.broadcast_to(n_eff, (b_, h_, n_)))
 
 
+@pytest.mark.parametrize("kw", [
+    dict(batch=1, heads_q=2, heads_kv=2, seq_len=64 * 16 + 37, head_dim=64, top_k=8),
+    dict(batch=1, heads_q=8, heads_kv=2, seq_len=64 * 12, head_dim=128, top_k=4, qkv_std=0.5),
+])
+def test_separate_scoring_query(kw):
+    """Q-Cal interface: summaries, select with q_score, attend_selected with q."""
+    inp = prefill_inputs(dtype="bf16", seed=31, **kw)
+    g = torch.Generator().manual_seed(32)
+    q_score = torch.randn(inp.q.shape, generator=g).to(torch.bfloat16)
+    out, idx = hils.attend(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.landmark.cuda(), kw["top_k"],
+                           q_score=q_score.cuda(), return_idx=True)
+    torch.cuda.synchronize()
+    ref = O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, kw["top_k"], q_score=q_score)
+    gi = idx.cpu().numpy()
+    check_indices(gi, ref["key"], kw["top_k"])
+    want = ref["out"]
+    if not np.array_equal(gi, ref["idx"]):
+        # near-tie rows: the oracle fused over the GPU's selection
+        want = O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, kw["top_k"], q_score=q_score,
+                         forced_idx=gi)["out"]
+    check_close(_np(out), want, True)
+
+
 def _rows_sample(n, rng, count=40):
     edge = [0, 1, 63, 64, 65, 127, 128, n // 2, n - 65, n - 64, n - 2, n - 1]
     return np.unique(np.concatenate([edge, rng.integers(0, n, count)]))
@@ -288,3 +311,55 @@ def test_bad_page_ids_are_flagged_not_faulted():
     assert call.device_status() == 0          # reading clears the word
     call(di.q.to(dev), kp, vp, kbar, hb, di.block_table.to(dev), di.seq_lens.to(dev))
     assert call.device_status() == 0
+
+
+# --------------------------------------------------------------------------- compact (bf16) summary cache
+@pytest.mark.parametrize("kw", [
+    dict(batch=5, heads_q=4, heads_kv=2, seq_len=0, head_dim=64, top_k=4, seq_lens=[1, 64, 65, 300, 1000]),
+    dict(batch=2, heads_q=16, heads_kv=16, seq_len=0, head_dim=64, top_k=16, seq_lens=[8192, 5000]),
+    dict(batch=2, heads_q=8, heads_kv=2, seq_len=0, head_dim=128, top_k=8, seq_lens=[3000, 64 * 40 + 1]),
+])
+def test_decode_with_bf16_summary_cache(kw):
+    """hils_summarize_paged_ex / hils_decode_ex with bf16 kbar pages.
+
+    The cache holds kbar rounded to bf16 (within half an ulp of the oracle's
+    fp32 summaries, plus fp32 summation error).  Scores from it carry at most
+    scale * 2^-8 * sum_e |q_e| |kbar_e| of rounding error, so the selection
+    must equal the oracle's wherever its K-th vs (K+1)-th gap exceeds twice
+    that bound; the outputs are compared with the oracle fused over the GPU's
+    selection, under the bf16 output tolerances.
+    """
+    K = kw["top_k"]
+    di = decode_inputs(dtype="bf16", seed=41, spare_pages=2, **kw)
+    P, g, B, d = di.k_pages.shape
+    h = di.landmark_pages.shape[1]
+    dev = "cuda"
+    kp, vp, lp = di.k_pages.to(dev), di.v_pages.to(dev), di.landmark_pages.to(dev)
+    ids = torch.arange(P, dtype=torch.int32, device=dev)
+    kbar16 = torch.zeros((P, h, d), dtype=torch.bfloat16, device=dev)
+    hb = torch.zeros((P, h), dtype=torch.float32, device=dev)
+    hils.summarize_paged(kp, lp, ids, kbar16, hb)
+    kbar32 = torch.zeros((P, h, d), dtype=torch.float32, device=dev)
+    hils.summarize_paged(kp, lp, ids, kbar32, torch.zeros_like(hb))
+    # the compact cache is the fp32 summary rounded to bf16
+    assert torch.equal(kbar16, kbar32.to(torch.bfloat16))
+    out, idx = hils.decode(di.q.to(dev), kp, vp, kbar16, hb, di.block_table.to(dev), di.seq_lens.to(dev), K,
+                           return_idx=True)
+    torch.cuda.synchronize()
+    scale = 1.0 / np.sqrt(d)
+    grp = h // g
+    q64 = di.q.double().numpy()
+    kb = kbar32.double().cpu().numpy()
+    for b in range(kw["batch"]):
+        for gsel in range(g):
+            q, kps, vps, lps, bt, sl = _slice_for_oracle(di, b, gsel)
+            ref = O.decode(q, kps, vps, lps, bt, sl, K)
+            gi = idx[b, gsel].cpu().numpy()
+            if sl[0] > 64:
+                pages = di.block_table[b].numpy()[: (sl[0] - 1) // 64]
+                bound = max(
+                    float((np.abs(q64[b, gsel * grp + hh])[None] * np.abs(kb[pages, gsel * grp + hh])).sum(-1).max())
+                    for hh in range(grp)) * scale * 2.0 ** -8
+                check_indices(gi[None], ref["key"][0][0][None], K, gap=2 * bound + 1e-3)
+            want = _forced_decode(q, kps, vps, lps, bt, sl, gi) if sl[0] > 64 else ref["out"][0]
+            check_close(_np(out[b, gsel * grp:(gsel + 1) * grp]), want, True)

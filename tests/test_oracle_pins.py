@@ -355,3 +355,46 @@ def test_decode_matches_prefill_rows():
         dec = O.decode(q[:, :, t], kp, vp, lp, bt, [t + 1] * b, K)
         assert np.allclose(dec["out"], pre["out"][:, :, t], atol=1e-12, rtol=0)
         assert np.array_equal(dec["idx"], pre["idx"][:, :, t])
+
+
+# --- separate scoring query (notes section 5.4, the Q-Cal interface) -------
+def test_scoring_query_equal_to_q_changes_nothing():
+    r = _rng(21)
+    b, h, g, n, d, B, K = 1, 4, 2, 300, 16, 64, 2
+    q, k, v = (r.standard_normal((b, x, n, d)) for x in (h, g, g))
+    lm = r.standard_normal((b, h, n // B, d))
+    a = O.forward(q, k, v, lm, B, K)
+    c = O.forward(q, k, v, lm, B, K, q_score=q.copy())
+    assert np.array_equal(a["idx"], c["idx"])
+    assert np.allclose(a["out"], c["out"], atol=0, rtol=0)
+
+
+def test_zero_scoring_query_selects_by_entropy_alone():
+    # shat = 0 . kbar + H_c = H_c: the selection is the top K of H (group max, lower index on ties)
+    r = _rng(22)
+    b, h, g, n, d, B, K = 1, 4, 2, 640, 8, 64, 3
+    q, k, v = (r.standard_normal((b, x, n, d)) for x in (h, g, g))
+    lm = 3.0 * r.standard_normal((b, h, n // B, d))
+    res = O.forward(q, k, v, lm, B, K, q_score=np.zeros_like(q))
+    _, hb = O.summarize(k, lm, B)
+    grp = h // g
+    for gi in range(g):
+        hmax = hb[0, gi * grp:(gi + 1) * grp].max(axis=0)
+        for i in range(0, n, 37):
+            cand = i // B
+            want = sorted(range(cand), key=lambda c: (-hmax[c], c))[:K]
+            got = [int(c) for c in res["idx"][0, gi, i] if c >= 0]
+            assert got == want
+
+
+def test_scoring_query_of_rows_without_candidates_is_unused():
+    r = _rng(23)
+    b, h, g, n, d, B, K = 1, 2, 2, 256, 16, 64, 2
+    q, k, v = (r.standard_normal((b, x, n, d)) for x in (h, g, g))
+    lm = r.standard_normal((b, h, n // B, d))
+    qs = r.standard_normal((b, h, n, d))
+    a = O.forward(q, k, v, lm, B, K, q_score=qs)
+    qs2 = qs.copy()
+    qs2[:, :, :B] = 1e3 * r.standard_normal((b, h, B, d))  # chunk 0 has no candidate chunk
+    c = O.forward(q, k, v, lm, B, K, q_score=qs2)
+    assert np.array_equal(a["out"], c["out"]) and np.array_equal(a["idx"], c["idx"])
