@@ -51,10 +51,10 @@ constexpr uint32_t kOwnFlag = 0x80000000u;
 
 template <int D>
 struct TcCfg {
-  static constexpr int NS = D == 64 ? 3 : 1;         // operand stages
-  static constexpr int NP = D == 64 ? 3 : 1;         // S / P slots (TMEM)
-  static constexpr int NO = D == 64 ? 3 : 2;         // P.V output slots (TMEM), >= NS
-  static constexpr int kRows = D == 64 ? 384 : 256;  // target rows (QB * G) per CTA
+  static constexpr int NS = D == 64 ? 2 : 1;         // operand stages
+  static constexpr int NP = D == 64 ? 2 : 1;         // S / P slots (TMEM)
+  static constexpr int NO = 2;                       // P.V output slots (TMEM), >= NS
+  static constexpr int kRows = D == 64 ? 512 : 256;  // target rows (QB * G) per CTA: more rows, fuller buckets
   static constexpr uint32_t kTmemCols = 512;  // NP S/P slots of 64 + NO output slots of D
   static constexpr uint32_t kStageA = 128 * D * 2, kStageK = 64 * D * 2, kStageV = 64 * D * 2;
   static constexpr uint32_t kStage = kStageA + kStageK + kStageV;
