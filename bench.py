@@ -63,10 +63,10 @@ def decode_bytes(cfg, summary_bytes=4):
 # profiles/).  Reported only while the kernel's sources are the ones it was taken on.
 ATTEND_TRAFFIC = {
     "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc.cu":
-                "c8500ff5a6374bea5ab48e689ed9ce21b7a8493011b381219bf932f260a03478",
+                "e68bab984477a65167cf7b4b8a1670c4fa61deed6de76f0149b5bb4b63fc3444",
                 "chunk_wise_hierarchical_b200/csrc/tc_util.cuh":
                 "2c8199fc4ff66b314758faa3af3800696b99b5856f4f2dcdf03a90bd6e6727b6"},
-    "bytes": 269144832 + 54669824,
+    "bytes": 277194752 + 55144192,
 }
 
 
