@@ -300,6 +300,41 @@ def run_prefill(args, ws_world, rank, local):
                 launches_per_step=3)
 
 
+def run_prefill_gqa(dev, steps=5, warmup=3):
+    """The 7B-shaped GQA prefill (b1 h32 g8 N32768 d128 K32): per-stage device times and
+    TFLOP/s of the same algorithmic FLOP count, reported beside the headline step."""
+    import chunk_wise_hierarchical_b200 as hils
+    cfg = CONFIGS["prefill_7b_gqa"]
+    inp = prefill_inputs(seed=0, device=dev, **cfg)
+    q, k, v, lm = inp.q, inp.k, inp.v, inp.landmark
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    K = cfg["top_k"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    for it in range(warmup + steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record()
+        kbar, hb = hils.summarize(k, lm)
+        ev[1].record()
+        idx, sc = hils.select(q, kbar, hb, K, g)
+        ev[2].record()
+        hils.attend_selected(q, k, v, idx, sc)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if it >= warmup:
+            times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(3)])
+    med = [statistics.median(t[i] for t in times) for i in range(3)]
+    flops = algorithmic_flops(b, h, n, d, K)
+    return {"workload": "prefill_7b_gqa: batch 1, 32 query heads / 8 KV heads, N 32768, d 128, top-k 32, bf16",
+            "ms_per_step": round(sum(med), 4),
+            "stage_ms": {"summarize": round(med[0], 4), "select": round(med[1], 4), "attend_selected": round(med[2], 4)},
+            "tflops": round(flops / (sum(med) * 1e-3) / 1e12, 3),
+            "attend_tflops": round(flops / (med[2] * 1e-3) / 1e12, 3),
+            "timing": "CUDA events per stage, median of %d steps, L2 flushed between steps" % steps}
+
+
 # ---------------------------------------------------------------------------- decode (ours)
 def run_decode(name, n_caches, dev, reps=50):
     """Decode step time for the fp32 summary cache and for the compact bf16 one, on the
@@ -376,6 +411,7 @@ def run_ours(args):
                                              "frac_hbm": round(r["gbs"] / hbm, 4)} for k, r in dec.items()}}))
         return
     pre = run_prefill(args, ws_world, rank, local)
+    gqa = run_prefill_gqa(torch.device("cuda", local)) if not args.no_gqa else None
     cpu = cpu_baseline(args.cpu_seconds) if (rank == 0 and ws_world == 1 and not args.no_cpu) else None
     if ws_world > 1:
         torch.distributed.barrier()
@@ -415,6 +451,8 @@ def run_ours(args):
         "gpu_launches": pre["launches_per_step"] * args.steps,
         "clocks": pre["clocks"],
     }
+    if gqa:
+        line["prefill_7b_gqa"] = gqa
     if dec:
         line["decode"] = {
             k: {"tok_s": round(r["tok_s"], 1), "us_per_step": round(r["ms"] * 1e3, 2),
@@ -466,6 +504,7 @@ def main():
     ap.add_argument("--decode-only", action="store_true", help="time only the decode configurations")
     ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-gqa", action="store_true", help="skip the 7B-shaped GQA prefill line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the attention kernel from an ncu capture")

@@ -51,10 +51,10 @@ constexpr uint32_t kOwnFlag = 0x80000000u;
 
 template <int D>
 struct TcCfg {
-  static constexpr int NS = D == 64 ? 2 : 1;         // operand stages
-  static constexpr int NP = D == 64 ? 2 : 1;         // S / P slots (TMEM)
+  static constexpr int NS = 2;                       // operand stages
+  static constexpr int NP = 2;                       // S / P slots (TMEM)
   static constexpr int NO = 2;                       // P.V output slots (TMEM), >= NS
-  static constexpr int kRows = D == 64 ? 512 : 256;  // target rows (QB * G) per CTA: more rows, fuller buckets
+  static constexpr int kRows = D == 64 ? 512 : 128;  // target rows (QB * G) per CTA: more rows, fuller buckets
   static constexpr uint32_t kTmemCols = 512;  // NP S/P slots of 64 + NO output slots of D
   static constexpr uint32_t kStageA = 128 * D * 2, kStageK = 64 * D * 2, kStageV = 64 * D * 2;
   static constexpr uint32_t kStage = kStageA + kStageK + kStageV;
@@ -62,7 +62,7 @@ struct TcCfg {
 };
 
 struct TcSmem {
-  uint32_t stage, o, list, off, items, rowm, rowz, total;
+  uint32_t stage, o, list, off, items, rowm, rowz, cur, total;
 };
 
 __host__ __device__ inline uint32_t align_to(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -84,6 +84,7 @@ __host__ __device__ inline TcSmem tc_layout(int G, int qb, int K, int n_cand) {
   L.items = off; off = align_to(off + (uint32_t)max_items(G, qb, K, n_cand) * 4, 16);
   L.rowm = off; off += (uint32_t)qb * G * 4;
   L.rowz = off; off += (uint32_t)qb * G * 4;
+  L.cur = off; off += (uint32_t)(n_cand + 1) * 4;  // scatter cursors of the bucket sort
   L.total = align_to(off, 16);
   return L;
 }
@@ -244,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   __syncthreads();
   const int n_entries = block_exclusive_scan(s_off, n_cand, s_wsum);
   const int n_sel_items = block_exclusive_scan(s_toff, n_cand, s_wsum);
-  // cursors for the scatter: a copy of the offsets in the per-row array (rows > n_cand)
-  int* cur = reinterpret_cast<int*>(s_rowm);
+  // cursors for the scatter: a copy of the offsets
+  int* cur = reinterpret_cast<int*>(sm + L.cur);
   for (int c = tid; c < n_cand; c += kThreads) cur[c] = s_off[c];
   if (tid == 0) s_off[n_cand] = n_entries;
   __syncthreads();
@@ -739,7 +740,6 @@ static int pick_qb(int G, int K, int N, size_t* smem_out) {
   int qb = TcCfg<D>::kRows / G;
   const int n_cand_max = N / kChunk;
   for (; qb >= 16; qb >>= 1) {
-    if (qb * G < n_cand_max + 1) continue;  // the scatter cursors borrow the per-row array
     const TcSmem L = tc_layout<D>(G, qb, K, n_cand_max);
     const size_t need = (size_t)L.total + 1024;
     if (need <= 227 * 1024 - 1024) {  // leave room for the static shared variables
