@@ -138,6 +138,132 @@ __global__ void select_simt_kernel(SelectArgs a, int qt) {
   }
 }
 
+// Register variant for K <= 32: one thread per (query, head) -- thread t takes query
+// t / G and head t % G of its KV group, so a thread holds one d-row of q (shared
+// memory, padded rows) and computes its head's scores; the group's max comes from
+// shuffles over its G consecutive lanes.  Every lane of a group keeps the same sorted
+// list of the best KP keys in registers, plus its own head's score of each listed
+// chunk (shifted together with the keys).
+template <int KP>
+__device__ __forceinline__ void sorted_insert2(unsigned long long (&L)[KP], float (&S)[KP], unsigned long long x,
+                                               float sx) {
+#pragma unroll
+  for (int j = KP - 1; j > 0; --j) {
+    const bool above_prev = x > L[j - 1];
+    const bool above_here = x > L[j];
+    L[j] = above_prev ? L[j - 1] : (above_here ? x : L[j]);
+    S[j] = above_prev ? S[j - 1] : (above_here ? sx : S[j]);
+  }
+  if (x > L[0]) {
+    L[0] = x;
+    S[0] = sx;
+  }
+}
+
+template <typename T, int D, int G, int KP>
+__global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
+  constexpr int QT = 128 / G;  // queries per CTA
+  constexpr int QS = D + 1;    // padded q row (floats)
+  constexpr int KS = D + 1;    // padded summary row
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qS = reinterpret_cast<float*>(smem_raw);  // [128][QS]
+  float* kbS = qS + 128 * QS;                      // [kSelCT][G][KS]
+  float* hbS = kbS + kSelCT * G * KS;              // [kSelCT][G]
+  const int t = threadIdx.x, lane = t & 31;
+  const int hh = t % G, qo = t / G;
+  const int K = a.top_k;
+  const int n_qtiles = (a.n + QT - 1) / QT;
+  const int qtile = blockIdx.x % n_qtiles;
+  const int gi = (blockIdx.x / n_qtiles) % a.g;
+  const int bi = blockIdx.x / (n_qtiles * a.g);
+  const int i = qtile * QT + qo;
+  const bool active = i < a.n;
+  const int n_cand = active ? min(i / kChunk, a.n_chunks) : 0;
+  const size_t head = (size_t)bi * a.h + gi * G + hh;
+  {
+    const T* qrow = static_cast<const T*>(a.q) + (head * a.n + (active ? i : 0)) * D;
+    for (int e = 0; e < D; e += 4) {
+      const float4 v = active ? load4(qrow + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float* dst = qS + t * QS + e;
+      dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+    }
+  }
+  const int last_i = min(a.n - 1, qtile * QT + QT - 1);
+  const int tile_cand = min(last_i / kChunk, a.n_chunks);
+  unsigned long long L[KP];
+  float Sc[KP];
+#pragma unroll
+  for (int s = 0; s < KP; ++s) {
+    L[s] = 0ull;  // below every real key
+    Sc[s] = -INFINITY;
+  }
+  for (int c0 = 0; c0 < tile_cand; c0 += kSelCT) {
+    __syncthreads();
+    for (int x = t; x < kSelCT * G * D; x += blockDim.x) {
+      const int cc = x / (G * D), h2 = (x / D) % G, e = x % D;
+      const int c = c0 + cc;
+      kbS[(cc * G + h2) * KS + e] =
+          c < a.n_chunks ? a.kbar[(((size_t)bi * a.h + gi * G + h2) * a.n_chunks + c) * D + e] : 0.f;
+    }
+    for (int x = t; x < kSelCT * G; x += blockDim.x) {
+      const int c = c0 + x / G, h2 = x % G;
+      hbS[x] = c < a.n_chunks ? a.hbias[((size_t)bi * a.h + gi * G + h2) * a.n_chunks + c] : 0.f;
+    }
+    __syncthreads();
+    float acc[kSelCT];
+#pragma unroll
+    for (int cc = 0; cc < kSelCT; ++cc) acc[cc] = 0.f;
+    const float* qr = qS + t * QS;
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) {
+      const float qe = qr[e];
+#pragma unroll
+      for (int cc = 0; cc < kSelCT; ++cc) acc[cc] = fmaf(qe, kbS[(cc * G + hh) * KS + e], acc[cc]);
+    }
+#pragma unroll
+    for (int cc = 0; cc < kSelCT; ++cc) {
+      const int c = c0 + cc;
+      const float own = fmaf(acc[cc], a.scale, hbS[cc * G + hh]);
+      float best = own;
+#pragma unroll
+      for (int o = 1; o < G; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+      if (c < n_cand) {
+        const unsigned long long key = pack_key(best, c);
+        if (key > L[KP - 1]) sorted_insert2(L, Sc, key, own);
+      }
+    }
+  }
+  (void)lane;
+  if (!active) return;
+  int32_t* idx_out = a.idx + (((size_t)bi * a.g + gi) * a.n + i) * K;
+  float* sc_out = a.score ? a.score + (head * a.n + i) * K : nullptr;
+#pragma unroll
+  for (int s = 0; s < KP; ++s) {
+    if (s < K) {
+      const bool have = L[s] != 0ull;
+      if (hh == 0) idx_out[s] = have ? key_chunk(L[s]) : -1;
+      if (sc_out) sc_out[s] = have ? Sc[s] : -INFINITY;
+    }
+  }
+}
+
+static size_t group_smem(int G, int D) {
+  return ((size_t)128 * (D + 1) + (size_t)kSelCT * G * (D + 1) + kSelCT * G) * 4;
+}
+
+template <typename T, int D, int G, int KP>
+static cudaError_t launch_group(const SelectArgs& a, cudaStream_t st) {
+  const size_t smem = group_smem(G, D);
+  cudaError_t e = cudaFuncSetAttribute(select_group_kernel<T, D, G, KP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  constexpr int QT = 128 / G;
+  const long long blocks = (long long)((a.n + QT - 1) / QT) * a.g * a.b;
+  if (blocks == 0) return cudaSuccess;
+  select_group_kernel<T, D, G, KP><<<(unsigned)blocks, 128, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 static size_t select_smem(int qt, int G, int D, int K) {
   size_t f = (size_t)qt * (G * D + 1) + kSelCT * G * D + ((kSelCT * G + 1) & ~1);
   return f * 4 + (size_t)K * qt * 8 + (size_t)K * G * qt * 4;
@@ -158,13 +284,20 @@ static cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <typename T, int D, int G>
+static cudaError_t launch_by_k(const SelectArgs& a, cudaStream_t st) {
+  if (a.top_k <= 16) return launch_group<T, D, G, 16>(a, st);
+  if (a.top_k <= 32) return launch_group<T, D, G, 32>(a, st);
+  return launch_select<T, D, G>(a, st);  // K up to 64: lists in shared memory
+}
+
 template <typename T, int D>
 static cudaError_t select_by_group(const SelectArgs& a, cudaStream_t st) {
   switch (a.h / a.g) {
-    case 1: return launch_select<T, D, 1>(a, st);
-    case 2: return launch_select<T, D, 2>(a, st);
-    case 4: return launch_select<T, D, 4>(a, st);
-    case 8: return launch_select<T, D, 8>(a, st);
+    case 1: return launch_by_k<T, D, 1>(a, st);
+    case 2: return launch_by_k<T, D, 2>(a, st);
+    case 4: return launch_by_k<T, D, 4>(a, st);
+    case 8: return launch_by_k<T, D, 8>(a, st);
   }
   return cudaErrorInvalidValue;
 }
