@@ -105,3 +105,19 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 64, 64)
     with pytest.raises((ValueError, RuntimeError)):
         hils.attend(q, q, q, torch.zeros(1, 1, 1, 64), top_k=1)
+
+
+def test_summary_dtype_validation():
+    lib = hils.lib()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below fails validation first
+    s_bf16 = _shape(dtype=1)
+    s_f32 = _shape(dtype=0)
+    # unknown summary dtype
+    assert lib.hils_summarize_paged_ex(ctypes.byref(s_bf16), fake, fake, fake, 4, 4, fake, 7, fake, None) == 1
+    assert lib.hils_decode_ex(ctypes.byref(s_bf16), fake, fake, fake, fake, 7, fake, fake, 1, fake, 4, fake,
+                              None, fake, 1 << 30, None) == 1
+    # a bf16 summary cache needs a bf16 model
+    assert lib.hils_summarize_paged_ex(ctypes.byref(s_f32), fake, fake, fake, 4, 4, fake, 1, fake, None) == 2
+    assert lib.hils_decode_ex(ctypes.byref(s_f32), fake, fake, fake, fake, 1, fake, fake, 1, fake, 4, fake,
+                              None, fake, 1 << 30, None) == 2
