@@ -63,10 +63,10 @@ def decode_bytes(cfg, summary_bytes=4):
 # profiles/).  Reported only while the kernel's sources are the ones it was taken on.
 ATTEND_TRAFFIC = {
     "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc.cu":
-                "e68bab984477a65167cf7b4b8a1670c4fa61deed6de76f0149b5bb4b63fc3444",
+                "4c6a1f6ec5766feac0161f8b1769ae25079562316b41a89b41a0a945490a6fe8",
                 "chunk_wise_hierarchical_b200/csrc/tc_util.cuh":
                 "2c8199fc4ff66b314758faa3af3800696b99b5856f4f2dcdf03a90bd6e6727b6"},
-    "bytes": 277194752 + 55144192,
+    "bytes": 276958976 + 57682688,
 }
 
 
