@@ -63,7 +63,7 @@ def decode_bytes(cfg, summary_bytes=4):
 # profiles/).  Reported only while the kernel's sources are the ones it was taken on.
 ATTEND_TRAFFIC = {
     "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc.cu":
-                "4c6a1f6ec5766feac0161f8b1769ae25079562316b41a89b41a0a945490a6fe8",
+                "7d38efcfbbc3491a04b890039c80d3d548f03906078c602df6d85e34c43e963a",
                 "chunk_wise_hierarchical_b200/csrc/tc_util.cuh":
                 "2c8199fc4ff66b314758faa3af3800696b99b5856f4f2dcdf03a90bd6e6727b6"},
     "bytes": 276958976 + 57682688,

@@ -5,14 +5,15 @@
 //
 // Work decomposition ("row owner, chunk buckets").  One CTA owns a block of QB
 // consecutive queries of one (sequence, KV head) and all G query heads of the
-// group: R = QB*G rows whose fp32 output accumulators stay in shared memory
-// for the whole CTA.  The CTA buckets its rows' selections by chunk (counting
-// sort in shared memory) and turns them into a list of work items: 128-row
-// tiles of (own chunk | selected chunk c, rows).  Per item
-//     S = Q_tile K_c^T          (tcgen05, M=128 N=64, S in TMEM)
-//     P_j = exp(x_j - m)        (registers -> bf16 shared memory)
-//     O_tile = P V_c            (tcgen05, M=128 N=d, TMEM)
-//     O[row] (=|+=) f * O_tile[row]   (shared memory)
+// group: R = QB*G rows (512 for d = 64, 128 for d = 128) whose fp32 output
+// accumulators stay in shared memory for the whole CTA.  The CTA buckets its
+// rows' selections by chunk (counting sort in shared memory) and turns them into
+// a list of work items: 128-row tiles of (own chunk | selected chunk c, rows).
+// Per item
+//     S = Q_tile K_c^T              (tcgen05, M=128 N=64, S in TMEM)
+//     P_j = f * exp(x_j - m)        (registers -> bf16, over S's TMEM columns)
+//     O_tile = P V_c                (tcgen05, A = P from TMEM, M=128 N=d, TMEM)
+//     O[row] (=|+=) O_tile[row]     (shared memory)
 // so every (row, chunk) pair contributes its final weighted term and no
 // partial result leaves the SM.  For a selected chunk f = exp(shat - M)/(Z' l);
 // for the own chunk f = exp(m - M)/Z', where the own item completes the
@@ -24,12 +25,11 @@
 //               ring of operand stages; a stage's Q/K half is reused once S has run
 //   warp 1      producer (one thread): TMA load of V_c, released after P.V
 //   warp 2      MMA issuer (one thread): an event loop issuing S(i) and P.V(j)
-//               as their inputs become ready; tcgen05.commit signals the rest
+//               as their inputs become ready; one tcgen05.commit per MMA group
 //   warps 4-11  two softmax warpgroups taking alternate items: TMEM ->
-//               registers -> P = exp(x - m) (bf16, swizzled smem) and the row's
-//               output multiplier
-//   warps 12-15 epilogue warpgroup: TMEM -> O_tile * multiplier -> shared-memory
-//               accumulators
+//               registers -> P (scaled by the row's fusion factor) -> TMEM
+//   warps 12-15 epilogue warpgroup: TMEM -> registers -> shared-memory
+//               accumulators (32-column halves, the next load overlapping)
 // Rows outside a tile's count are computed and ignored (padding of the
 // 128-row MMA).  Summation over chunks runs in chunk-index order, so results
 // do not depend on the order of rows inside a bucket.
@@ -110,9 +110,6 @@ __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
       : "memory");
   return out != 0;
 }
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
 }
@@ -190,8 +187,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   float* s_rowz = reinterpret_cast<float*>(sm + L.rowz);
 
   const __nv_bfloat16* qg = a.q + ((size_t)bi * a.h + head0) * N * D;
-  const __nv_bfloat16* kg = a.k + ((size_t)bi * a.g + gi) * N * D;
-  const __nv_bfloat16* vg = a.v + ((size_t)bi * a.g + gi) * N * D;
   const int32_t* idxg = a.idx + ((size_t)bi * a.g + gi) * N * K;
   const float* sselg = a.ssel + ((size_t)bi * a.h + head0) * N * K;
 
