@@ -1,7 +1,11 @@
 """Builds libhils.so (all CUDA sources under csrc/) for sm_100a with nvcc.
 
 Usage: python -m chunk_wise_hierarchical_b200.build [--force]
-The library is written next to this file so that it travels with the package.
+Each source is compiled to its own object, in parallel; decode_slice.cu is compiled once
+per (element type, head dim, group size) slice of the decode kernels.  The objects are
+then linked into one shared library, written next to this file so that it travels with
+the package.  The stamp beside it hashes the sources by their paths relative to the
+package, so a copy of the tree at another path reuses the library.
 """
 from __future__ import annotations
 
@@ -11,6 +15,8 @@ import os
 import shutil
 import subprocess
 import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
@@ -22,8 +28,11 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "--std=c++17",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-    "-shared", "-Xptxas", "-warn-spills",
+    "-Xptxas", "-warn-spills",
 ]
+SLICED = "decode_slice.cu"
+# (element type: 0 fp32 / 1 bf16, head dim, group size) of each decode slice
+DECODE_SLICES = [(t, d, g) for t in (1, 0) for d in (64, 128) for g in (1, 2, 4, 8)]
 
 
 def _sources():
@@ -34,10 +43,11 @@ def _digest():
     h = hashlib.sha256()
     files = _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "hils.h")]
     for f in files:
-        h.update(f.encode())
+        h.update(os.path.relpath(f, os.path.dirname(HERE)).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
     h.update(" ".join(NVCC_FLAGS).encode())
+    h.update(repr(DECODE_SLICES).encode())
     return h.hexdigest()
 
 
@@ -55,10 +65,34 @@ def build(force: bool = False, verbose: bool = False) -> str:
             if f.read().strip() == dig:
                 return LIB
     tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *_sources()]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    with tempfile.TemporaryDirectory(prefix="hils_build_") as objdir:
+        jobs = []
+        for src in _sources():
+            name = os.path.splitext(os.path.basename(src))[0]
+            if os.path.basename(src) == SLICED:
+                for t, d, g in DECODE_SLICES:
+                    defs = [f"-DHILS_DECODE_T={t}", f"-DHILS_DECODE_D={d}", f"-DHILS_DECODE_G={g}"]
+                    jobs.append((src, defs, os.path.join(objdir, f"{name}_{t}_{d}_{g}.o")))
+            else:
+                jobs.append((src, [], os.path.join(objdir, name + ".o")))
+
+        def compile_one(job):
+            src, defs, obj = job
+            cmd = [nvcc_path(), *NVCC_FLAGS, *defs, "-I", INCLUDE, "-c", "-o", obj, src]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            return subprocess.run(cmd).returncode, src, defs
+
+        # the decode slices (bf16 ones first) are the slowest objects: start them first
+        jobs.sort(key=lambda j: os.path.basename(j[0]) != SLICED)
+        with ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as pool:
+            results = list(pool.map(compile_one, jobs))
+        failed = [(src, defs) for rc, src, defs in results if rc != 0]
+        if failed:
+            raise RuntimeError(f"nvcc failed on {failed}")
+        link = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                "-o", tmp, *[obj for _, _, obj in jobs]]
+        subprocess.run(link, check=True)
     os.replace(tmp, LIB)
     with open(STAMP, "w") as f:
         f.write(dig)

@@ -1,0 +1,674 @@
+// Single-token decode over a paged chunk cache (HiLS notes, sections 5.2-5.4,
+// applied to the newest query of each sequence).  Two HBM-bound kernels,
+// chained with programmatic dependent launch:
+//
+// 1. decode_scan_kernel -- grid (sequence, range of candidate chunks).  Each CTA
+//    reads the cached summaries of its range page by page, all heads at once (a
+//    page's [h][d] fp32 block is contiguous), scores them (q . kbar * scale + H, GQA
+//    max over the group's heads) and, one warp per KV head, sorts the range's keys
+//    and writes its best K.  The last CTA of the sequence -- an atomic ticket; no
+//    CTA waits on another -- merges the ranges' lists into the final Top-K and
+//    writes each head's own score of the selected chunks.
+// 2. decode_attend_kernel -- one warp per chunk (own chunk or one Top-K slot),
+//    all G heads sharing each K/V load, K and V staged in shared memory with
+//    cp.async.  The own chunk does not depend on the selection and is
+//    computed before the kernel waits for the scan grid.  Each warp writes
+//    its chunk's (max, sum, unnormalised output); the last CTA of the
+//    (sequence, KV head) fuses them with the inter-chunk softmax of notes
+//    section 5.3 (own chunk at its exact log-mass).
+// Tickets are reset by the CTA that consumes them, so both kernels can be
+// replayed (CUDA graphs) without clearing the workspace.
+#pragma once
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hils {
+
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kMaxRange = 256;          // candidate chunks per scan CTA, at most ...
+constexpr int kMinRange = 16;           // ... and at least
+constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B200
+constexpr int kMergeN = 256;            // keys one warp sorts at once in the fallback merge
+
+
+constexpr int kMaxListsPerLane = 4;
+
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
+// Descending bitonic sort of the warp's 32*E keys; element i lives in lane i / E,
+// register i % E.  All 32 lanes call it.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(unsigned long long (&v)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= E) {  // partner in lane ^ (j / E), same register
+        const int lj = j / E;
+        const bool lower = (lane & lj) == 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const bool desc = ((lane * E + e) & k) == 0;
+          const unsigned long long o = shfl_xor_u64(v[e], lj);
+          const bool keep_max = lower == desc;
+          v[e] = keep_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+        }
+      } else {  // partner in this lane, register e ^ j
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if ((e ^ j) > e) {
+            const bool desc = ((lane * E + e) & k) == 0;
+            const unsigned long long x = v[e], y = v[e ^ j];
+            const bool sw = desc ? x < y : x > y;
+            v[e] = sw ? y : x;
+            v[e ^ j] = sw ? x : y;
+          }
+        }
+      }
+    }
+  }
+}
+// Top-K of one KV head over this CTA's range: the key of chunk j is the max over the
+// group's heads of s_score[j][head] (a NaN, from a bad page, makes the key 0).  Writes
+// the K best keys (0 where the range has fewer) in descending order.
+template <int E, int G>
+__device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, int nc, int c_lo, int K,
+                                           unsigned long long* out) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int j = e * 32 + lane;  // any placement works: the keys are sorted next
+    unsigned long long key = 0;
+    if (j < nc) {
+      float best = -INFINITY;
+      bool bad = false;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float x = s_score[(size_t)j * H + gi * G + hh];
+        bad |= x != x;
+        best = fmaxf(best, x);
+      }
+      key = bad ? 0ull : pack_key(best, c_lo + j);
+    }
+    v[e] = key;
+  }
+  warp_sort_desc<E>(v);
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane * E + e;
+    if (i < K) out[i] = v[e];
+  }
+  for (int i = 32 * E + lane; i < K; i += 32) out[i] = 0ull;
+}
+
+// Scan: CTA per (sequence, range of chunks), all heads.  A page's summaries of all
+// heads, [h][d] fp32, are one contiguous block; thread t holds float4 t + 256 k of it
+// (FPT per thread), so each page is read with fully coalesced 16-byte loads, PB pages
+// in flight per thread.  Per (chunk, head) the dot with q is reduced over the d/4
+// lanes of the head row, scaled and biased by H into shared memory; then one warp per
+// KV head sorts the range's keys and writes its best K.  The last CTA of the sequence
+// (atomic ticket; no CTA waits on another) merges the ranges' lists.
+// Four CTAs per SM (64 registers a thread): a page gather's bandwidth grows with the
+// warps resident on the SM far more than with the loads each warp has in flight.
+// S: element type of the cached summaries (fp32, or bf16 for the compact cache).
+// MULTI: a page's block is narrower than the CTA, so one load step covers several pages.
+template <typename T, int D, int G, typename S, int FPT, bool MULTI>
+__global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) float s_score[];  // [range][h]; reused by the merge
+  __shared__ int s_page[kMaxRange];
+  __shared__ int s_last;
+  constexpr int EPP = 16 / (int)sizeof(S);       // summary elements per 16-byte piece
+  constexpr int QPR = D / EPP;                   // pieces per head row
+  // load steps per batch: 8 pages' worth of fp32 pieces per thread (bf16 pieces hold twice
+  // the elements, so half the steps keep the registers the same)
+  constexpr int PB = FPT >= 8 ? 1 : (8 / FPT) * 4 / EPP > 0 ? (8 / FPT) * 4 / EPP : 1;
+
+  pdl_launch_dependents();  // the attend grid may start its selection-independent prologue
+  const int t = threadIdx.x, warp = t >> 5;
+  const int split = blockIdx.x % a.nsplit;
+  const int bi = blockIdx.x / a.nsplit;
+  const int H = a.h, K = a.top_k, R = a.range;
+  const int c_lo = split * R;
+  const int32_t* bt = a.block_table + (size_t)bi * a.max_chunks;
+  const int L = a.seq_lens[bi];
+  const int own = L > 0 ? (L - 1) / kChunk : 0;
+  const int n_cand = min(own, a.max_chunks);
+  const int nc = max(0, min(n_cand, c_lo + R) - c_lo);
+  for (int x = t; x < nc; x += kScanThreads) s_page[x] = bt[c_lo + x];
+  // A page's summaries [h][d] are F 16-byte pieces.  When a page block is smaller than
+  // the CTA, one load step covers PPI pages (thread t: page t / F, piece t % F);
+  // otherwise thread t takes pieces t + 256 k of one page.
+  const int F = H * QPR;
+  const int PPI = MULTI ? kScanThreads / F : 1;
+  const int w = MULTI ? t / F : 0;
+  const int fl = MULTI ? t % F : t;
+  const bool tw = !MULTI || w < PPI;
+  float qf[FPT][EPP];
+#pragma unroll
+  for (int k = 0; k < FPT; ++k) {
+    const int f = fl + k * kScanThreads;
+    const T* qp = static_cast<const T*>(a.q) + ((size_t)bi * H + f / QPR) * D + (f % QPR) * EPP;
+#pragma unroll
+    for (int e = 0; e < EPP; ++e) qf[k][e] = tw && f < F ? to_f(qp[e]) : 0.f;
+  }
+  __syncthreads();
+
+  // Pages are processed in batches of PB load steps: the batch's loads are all in flight
+  // before the first is reduced.
+  const uint4* kb16 = reinterpret_cast<const uint4*>(a.kbar_pages);
+  struct Batch {
+    uint4 kv[PB][FPT];
+    float hv[PB][FPT];  // H of the lane's head (read by the lane that writes the score)
+    int pg[PB];
+  };
+  auto load = [&](Batch& B, int j0) {
+#pragma unroll
+    for (int u = 0; u < PB; ++u) {
+      const int j = j0 + u * PPI + w;
+      B.pg[u] = tw && j < nc ? s_page[j] : -1;
+      const bool ok = B.pg[u] >= 0 && B.pg[u] < a.n_pages;
+#pragma unroll
+      for (int k = 0; k < FPT; ++k) {
+        const int f = fl + k * kScanThreads;
+        B.kv[u][k] = ok && f < F ? __ldg(kb16 + (size_t)B.pg[u] * F + f) : make_uint4(0, 0, 0, 0);
+        B.hv[u][k] = ok && f < F && f % QPR == 0 ? __ldg(a.hbias_pages + (size_t)B.pg[u] * H + f / QPR) : 0.f;
+      }
+    }
+  };
+  auto reduce = [&](const Batch& B, int j0) {
+#pragma unroll
+    for (int u = 0; u < PB; ++u) {
+      const int j = j0 + u * PPI + w;
+#pragma unroll
+      for (int k = 0; k < FPT; ++k) {
+        const int f = fl + k * kScanThreads;
+        float x[EPP];
+        if constexpr (sizeof(S) == 2) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&B.kv[u][k]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 y = __bfloat1622float2(h2[i]);
+            x[2 * i] = y.x;
+            x[2 * i + 1] = y.y;
+          }
+        } else {
+          x[0] = __uint_as_float(B.kv[u][k].x); x[1] = __uint_as_float(B.kv[u][k].y);
+          x[2] = __uint_as_float(B.kv[u][k].z); x[3] = __uint_as_float(B.kv[u][k].w);
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) dot = fmaf(qf[k][e], x[e], dot);
+#pragma unroll
+        for (int o = QPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (tw && j < nc && f < F && f % QPR == 0) {
+          const int head = f / QPR, p = B.pg[u];
+          float sc = NAN;
+          if (p >= 0 && p < a.n_pages) sc = fmaf(dot, a.scale, B.hv[u][k]);
+          else set_error(a.err, kErrBadPage);
+          s_score[(size_t)j * H + head] = sc;
+        }
+      }
+    }
+  };
+  for (int j0 = 0; j0 < nc; j0 += PB * PPI) {
+    Batch bt_;
+    load(bt_, j0);
+    reduce(bt_, j0);
+  }
+  __syncthreads();
+
+  // per KV head: this range's best K
+  const int E = nc <= 32 ? 1 : nc <= 64 ? 2 : nc <= 128 ? 4 : 8;
+  for (int gi = warp; gi < a.g; gi += kScanWarps) {
+    unsigned long long* part = a.part_keys + (((size_t)bi * a.g + gi) * a.nsplit + split) * K;
+    switch (E) {
+      case 1: range_topk<1, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      case 2: range_topk<2, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      case 4: range_topk<4, G>(s_score, H, gi, nc, c_lo, K, part); break;
+      default: range_topk<8, G>(s_score, H, gi, nc, c_lo, K, part); break;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (t == 0) s_last = atomicAdd(a.scan_ticket + (size_t)bi * a.g, 1u) == (unsigned)(a.nsplit - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- last CTA of the sequence: per KV head, merge the ranges' lists ----
+  const int lane = t & 31;
+  const int n_all = a.nsplit * K;
+  // the selected keys of slots lane and lane + 32, in descending order (0: empty)
+  auto emit = [&](int gi, unsigned long long k0, unsigned long long k1) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int s = lane + 32 * r;
+      const unsigned long long key = r ? k1 : k0;
+      if (s < K) {
+        const int c = key ? (int)key_chunk(key) : -1;
+        a.idx[((size_t)bi * a.g + gi) * K + s] = c;
+        a.sel_page[((size_t)bi * a.g + gi) * K + s] = c >= 0 ? bt[c] : -1;
+        // G = 1: the selection key is the head's own score
+        if (G == 1) a.ssel[((size_t)bi * a.h + gi) * K + s] = key ? unorderable((uint32_t)(key >> 32)) : -INFINITY;
+      }
+    }
+  };
+  if (a.nsplit <= 32 * kMaxListsPerLane) {
+    // tournament: the lists are sorted, so each step is a warp max over the lists' heads
+    // (keys are unique: they carry the chunk index).  Lane l follows lists l, l + 32, ...
+    // straight from global memory, holding each list's head and the key after it, and
+    // fetching the next one as soon as a head is taken.
+    for (int gi = warp; gi < a.g; gi += kScanWarps) {
+      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
+      int pos[kMaxListsPerLane];
+      unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
+#pragma unroll
+      for (int m = 0; m < kMaxListsPerLane; ++m) {
+        const int l = lane + 32 * m;
+        const bool live = l < a.nsplit;
+        pos[m] = 0;
+        head[m] = live ? __ldcg(parts + (size_t)l * K) : 0ull;
+        next[m] = live && K > 1 ? __ldcg(parts + (size_t)l * K + 1) : 0ull;
+      }
+      unsigned long long res0 = 0ull, res1 = 0ull;
+      for (int s = 0; s < K; ++s) {
+        unsigned long long lb = head[0];
+#pragma unroll
+        for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
+        unsigned long long wb = lb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = shfl_xor_u64(wb, o);
+          wb = y > wb ? y : wb;
+        }
+        if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
+#pragma unroll
+        for (int m = 0; m < kMaxListsPerLane; ++m) {
+          if (head[m] == wb) {  // this lane's list m holds the winner: advance it
+            ++pos[m];
+            head[m] = next[m];
+            next[m] = pos[m] + 1 < K ? __ldcg(parts + (size_t)(lane + 32 * m) * K + pos[m] + 1) : 0ull;
+          }
+        }
+        if ((s & 31) == lane) {
+          if (s < 32) res0 = wb;
+          else res1 = wb;
+        }
+      }
+      emit(gi, res0, res1);
+    }
+  } else {
+    // running best K + the next slice of keys, sorted by the warp
+    for (int gi = warp; gi < a.g; gi += kScanWarps) {
+      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
+      constexpr int ME = kMergeN / 32;
+      unsigned long long v[ME];
+#pragma unroll
+      for (int e = 0; e < ME; ++e) v[e] = 0ull;
+      for (int start = 0; start < n_all; start += kMergeN - K) {
+        const int take = min(kMergeN - K, n_all - start);
+#pragma unroll
+        for (int e = 0; e < ME; ++e) {
+          const int i = lane * ME + e;
+          if (i >= K) v[e] = i - K < take ? __ldcg(parts + start + i - K) : 0ull;
+        }
+        warp_sort_desc<ME>(v);
+      }
+      // slot s sits in lane s / ME, register s % ME: move slots lane and lane + 32 here
+      unsigned long long k0 = 0ull, k1 = 0ull;
+#pragma unroll
+      for (int e = 0; e < ME; ++e) {
+        const unsigned long long x0 = __shfl_sync(0xffffffffu, (uint32_t)v[e], lane / ME) |
+                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), lane / ME) << 32);
+        const unsigned long long x1 = __shfl_sync(0xffffffffu, (uint32_t)v[e], (lane + 32) / ME) |
+                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), (lane + 32) / ME) << 32);
+        if (lane % ME == e) k0 = x0;
+        if ((lane + 32) % ME == e) k1 = x1;
+      }
+      emit(gi, k0, k1);
+    }
+  }
+  if constexpr (G > 1) {
+    __syncthreads();  // the selection written above is read back below
+    // each head's own score of the selected chunks: one warp per (KV head, slot, head)
+    for (int x = warp; x < a.g * K * G; x += kScanWarps) {
+      const int gi = x / (K * G), s = (x / G) % K, hh = x % G;
+      const int c = a.idx[((size_t)bi * a.g + gi) * K + s];
+      float sc = -INFINITY;
+      if (c >= 0) {
+        const int p = bt[c];
+        const S* kb = static_cast<const S*>(a.kbar_pages) + ((size_t)p * H + gi * G + hh) * D;
+        const T* qr = static_cast<const T*>(a.q) + ((size_t)bi * H + gi * G + hh) * D;
+        float acc = 0.f;
+#pragma unroll
+        for (int e = lane; e < D; e += 32) acc = fmaf(to_f(qr[e]), to_f(kb[e]), acc);
+        acc = warp_sum(acc);
+        sc = fmaf(acc, a.scale, __ldg(a.hbias_pages + (size_t)p * H + gi * G + hh));
+      }
+      if (lane == 0) a.ssel[((size_t)bi * H + gi * G + hh) * K + s] = sc;
+    }
+  }
+  if (t == 0) a.scan_ticket[(size_t)bi * a.g] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// Attention: one warp per half chunk (32 keys) of the own chunk or of a Top-K slot,
+// all G heads sharing each K/V load.  Lanes own keys for Q.K (each reads its key row)
+// and output columns for P.V (V rows are read across the lanes); nothing is staged,
+// so many warps fit per SM.  Each warp writes its half's (max, sum, unnormalised
+// output) per head; the last CTA of the (sequence, KV head) combines the halves of
+// each chunk and fuses the chunks with the inter-chunk softmax of notes section 5.3
+// (own chunk at its exact log-mass).
+constexpr int kAttWarps = 4;
+
+// Raw register types for one lane's share of a V row (CPL elements of T).
+template <int BYTES> struct RawT;
+template <> struct RawT<4> { using type = uint32_t; };
+template <> struct RawT<8> { using type = uint2; };
+template <> struct RawT<16> { using type = uint4; };
+
+template <typename T, int CPL>
+__device__ __forceinline__ void raw_to_f(const typename RawT<CPL * sizeof(T)>::type& r, float (&f)[CPL]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&r);
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < CPL / 2; ++i) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) f[i] = __uint_as_float(w[i]);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_row16(const T* src, float (&f)[16 / sizeof(T)]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(h[i]);
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  } else {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+  }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArgs a) {
+  constexpr int CPL = D / 32;                  // output columns per lane (adjacent)
+  constexpr int EPP = 16 / (int)sizeof(T);     // elements per 16-byte piece
+  constexpr int PPR = D / EPP;                 // pieces per key row
+  __shared__ __align__(16) float qS[G][D];
+  __shared__ float s_w[G][2 * (kMaxTopK + 1)];  // fusion weight of each half chunk, per head
+  __shared__ int s_last;
+
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int ngrp = a.att_ctas;
+  const int grp_i = blockIdx.x % ngrp;
+  const int gi = (blockIdx.x / ngrp) % a.g;
+  const int bi = blockIdx.x / (ngrp * a.g);
+  const int K = a.top_k;
+  const int n_items = 2 * (K + 1);             // item 2s + hf: slot s (0 own, s >= 1 Top-K s-1), half hf
+  const size_t part_stride = (size_t)G * (D + 2);
+  float* part = a.part_att + ((size_t)bi * a.g + gi) * (size_t)n_items * part_stride;
+  const int L = a.seq_lens[bi];
+  for (int x = t; x < G * D; x += blockDim.x)
+    qS[x / D][x % D] = to_f(static_cast<const T*>(a.q)[((size_t)bi * a.h + gi * G) * D + x]);
+  __syncthreads();
+
+  const int item = grp_i * kAttWarps + warp;
+  const int hf = item & 1;
+  auto run_item = [&](int c, int p, int nvalid) {
+    float* dst = part + (size_t)item * part_stride;
+    if (c >= 0 && (p < 0 || p >= a.n_pages)) set_error(a.err, kErrBadPage);
+    const int n_half = min(32, nvalid - 32 * hf);  // valid keys in this half
+    if (c < 0 || p < 0 || p >= a.n_pages || n_half <= 0) {
+      if (lane < G) dst[lane * (D + 2)] = -INFINITY;  // absent
+      return;
+    }
+    const size_t row0 = (((size_t)p * a.g + gi) * kChunk + 32 * hf) * D;
+    const T* kp = static_cast<const T*>(a.k_pages) + row0;
+    const T* vp = static_cast<const T*>(a.v_pages) + row0;
+    // Every load of the item is issued up front (its K row for Q.K, lane = key; the
+    // first VB rows of V for P.V, lane = output columns), so the item costs one memory
+    // round trip when VB covers the half.
+    using VRaw = typename RawT<CPL * sizeof(T)>::type;
+    constexpr int VB = CPL * sizeof(T) <= 4 ? 32 : 16;  // V rows per batch (registers)
+    const bool valid = lane < n_half;
+    uint4 kraw[PPR];
+#pragma unroll
+    for (int pc = 0; pc < PPR; ++pc)
+      kraw[pc] = valid ? *reinterpret_cast<const uint4*>(kp + (size_t)lane * D + pc * EPP) : make_uint4(0, 0, 0, 0);
+    VRaw vraw[VB];
+#pragma unroll
+    for (int u = 0; u < VB; ++u)
+      if (u < n_half) vraw[u] = *reinterpret_cast<const VRaw*>(vp + (size_t)u * D + lane * CPL);
+    float s[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) s[hh] = 0.f;
+#pragma unroll
+    for (int pc = 0; pc < PPR; ++pc) {
+      float f[EPP];
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[pc]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 x = __bfloat1622float2(h2[i]);
+          f[2 * i] = x.x;
+          f[2 * i + 1] = x.y;
+        }
+      } else {
+        f[0] = __uint_as_float(kraw[pc].x); f[1] = __uint_as_float(kraw[pc].y);
+        f[2] = __uint_as_float(kraw[pc].z); f[3] = __uint_as_float(kraw[pc].w);
+      }
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < EPP; ++e) s[hh] = fmaf(qS[hh][pc * EPP + e], f[e], s[hh]);
+    }
+    float pr[G], o[G][CPL];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const float x = valid ? s[hh] * a.scale : -INFINITY;
+      const float m = warp_max(x);
+      pr[hh] = valid ? expf(x - m) : 0.f;
+      const float l = warp_sum(pr[hh]);
+      if (lane == 0) {
+        dst[hh * (D + 2)] = m;
+        dst[hh * (D + 2) + 1] = l;
+      }
+#pragma unroll
+      for (int x2 = 0; x2 < CPL; ++x2) o[hh][x2] = 0.f;
+    }
+    // P.V over the rows in registers, then any further batches
+    for (int j0 = 0; j0 < n_half; j0 += VB) {
+      if (j0 > 0) {
+#pragma unroll
+        for (int u = 0; u < VB; ++u)
+          if (j0 + u < n_half) vraw[u] = *reinterpret_cast<const VRaw*>(vp + (size_t)(j0 + u) * D + lane * CPL);
+      }
+#pragma unroll
+      for (int u = 0; u < VB; ++u) {
+        if (j0 + u >= n_half) break;
+        float vj[CPL];
+        raw_to_f<T, CPL>(vraw[u], vj);
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float pj = __shfl_sync(0xffffffffu, pr[hh], (j0 + u) & 31);
+#pragma unroll
+          for (int x2 = 0; x2 < CPL; ++x2) o[hh][x2] = fmaf(pj, vj[x2], o[hh][x2]);
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int x2 = 0; x2 < CPL; ++x2) dst[hh * (D + 2) + 2 + lane * CPL + x2] = o[hh][x2];
+  };
+
+  // the own chunk does not depend on the selection: compute it before waiting
+  const int own = L > 0 ? (L - 1) / kChunk : 0;
+  if (item < 2 && L > 0)
+    run_item(own, own < a.max_chunks ? a.block_table[(size_t)bi * a.max_chunks + own] : -1, L - own * kChunk);
+  pdl_wait_primary();
+  if (item >= 2 && item < n_items && L > 0) {
+    const size_t slot = ((size_t)bi * a.g + gi) * K + (item >> 1) - 1;
+    run_item(a.idx[slot], a.sel_page[slot], kChunk);
+  }
+
+  __threadfence();
+  __syncthreads();
+  if (t == 0) s_last = atomicAdd(a.att_ticket + (size_t)bi * a.g + gi, 1u) == (unsigned)(ngrp - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  T* out = static_cast<T*>(a.out);
+  if (L <= 0) {
+    for (int x = t; x < G * D; x += blockDim.x) out[((size_t)bi * a.h + gi * G) * D + x] = from_f<T>(0.f);
+    if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
+    return;
+  }
+  // fusion weights, one warp per head: lane s handles slot s (3 rounds cover K + 1 <= 65 slots)
+  for (int hh = warp; hh < G; hh += kAttWarps) {
+    const float* sc_row = a.ssel + ((size_t)bi * a.h + gi * G + hh) * K;
+    float lg[3], ms[3], ls[3], mh[3][2];
+    bool ok[3];
+    float M = -INFINITY;
+#pragma unroll
+    for (int rr = 0; rr < 3; ++rr) {
+      const int sl = lane + 32 * rr;
+      ok[rr] = false;
+      lg[rr] = -INFINITY;
+      ms[rr] = -INFINITY;
+      ls[rr] = 0.f;
+      mh[rr][0] = mh[rr][1] = -INFINITY;
+      if (sl < K + 1) {
+        float lh[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float* pp = part + (size_t)(2 * sl + h2) * part_stride + hh * (D + 2);
+          mh[rr][h2] = __ldcg(pp);
+          lh[h2] = mh[rr][h2] != -INFINITY ? __ldcg(pp + 1) : 0.f;
+        }
+        ms[rr] = fmaxf(mh[rr][0], mh[rr][1]);
+        ok[rr] = ms[rr] != -INFINITY;
+        if (ok[rr]) {
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2)
+            if (mh[rr][h2] != -INFINITY) ls[rr] += lh[h2] * expf(mh[rr][h2] - ms[rr]);
+          lg[rr] = sl == 0 ? ms[rr] + logf(ls[rr]) : __ldcg(sc_row + sl - 1);
+        }
+      }
+      M = fmaxf(M, lg[rr]);
+    }
+    M = warp_max(M);
+    float z = 0.f;
+#pragma unroll
+    for (int rr = 0; rr < 3; ++rr) z += ok[rr] ? expf(lg[rr] - M) : 0.f;
+    const float Z = warp_sum(z);
+#pragma unroll
+    for (int rr = 0; rr < 3; ++rr) {
+      const int sl = lane + 32 * rr;
+      if (sl < K + 1) {
+        // own: exp(LSE_own - M)/Z * o/l = exp(m - M)/Z * o ; selected: exp(shat - M)/(Z l) * o,
+        // with the chunk's (m, l, o) combined from its halves (o_h rescaled by exp(m_h - m))
+        const float wsl = !ok[rr] ? 0.f : (sl == 0 ? expf(ms[rr] - M) / Z : expf(lg[rr] - M) / (Z * ls[rr]));
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+          s_w[hh][2 * sl + h2] = mh[rr][h2] == -INFINITY ? 0.f : wsl * expf(mh[rr][h2] - ms[rr]);
+      }
+    }
+  }
+  __syncthreads();
+  // weighted sum of the half-chunk outputs: thread = (head, column); the partials of a
+  // batch of items are all loaded before they are summed
+  constexpr int kFB = 16;
+  for (int x = t; x < G * D; x += blockDim.x) {
+    const int hh = x / D, col = x % D;
+    const float* pc = part + (size_t)hh * (D + 2) + 2 + col;
+    float acc = 0.f;
+    for (int it0 = 0; it0 < n_items; it0 += kFB) {
+      float v[kFB], w[kFB];
+#pragma unroll
+      for (int u = 0; u < kFB; ++u) {
+        const int it = it0 + u;
+        w[u] = it < n_items ? s_w[hh][it] : 0.f;
+        v[u] = w[u] != 0.f ? __ldcg(pc + (size_t)it * part_stride) : 0.f;  // absent halves were never written
+      }
+#pragma unroll
+      for (int u = 0; u < kFB; ++u) acc = fmaf(v[u], w[u], acc);
+    }
+    out[((size_t)bi * a.h + gi * G + hh) * D + col] = from_f<T>(acc);
+  }
+  if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
+}
+
+template <typename T, int D, int G, typename S, int FPT, bool MULTI = false>
+static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores
+  cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, S, FPT, MULTI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_scan_kernel<T, D, G, S, FPT, MULTI><<<(unsigned)a.b * a.nsplit, kScanThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int G, typename S>
+static cudaError_t launch_scan_by_width(const DecodeArgs& a, cudaStream_t st) {
+  const int f16 = a.h * D * (int)sizeof(S) / 16;  // 16-byte pieces per page of summaries
+  const int fpt = (f16 + kScanThreads - 1) / kScanThreads;
+  if (f16 < kScanThreads) return launch_scan<T, D, G, S, 1, true>(a, st);
+  return fpt <= 1 ? launch_scan<T, D, G, S, 1>(a, st)
+       : fpt <= 2 ? launch_scan<T, D, G, S, 2>(a, st)
+       : fpt <= 4 ? launch_scan<T, D, G, S, 4>(a, st)
+                  : launch_scan<T, D, G, S, 8>(a, st);
+}
+
+template <typename T, int D, int G>
+static cudaError_t launch_decode(DecodeArgs a, cudaStream_t st) {
+  const unsigned bg = (unsigned)a.b * a.g;
+  if (bg == 0) return cudaSuccess;
+  if (!decode_supported(a.h, D)) return cudaErrorInvalidValue;
+  if (a.top_k > 0) {
+    cudaError_t e;
+    if (a.kbar_bf16) {
+      if constexpr (sizeof(T) == 2) e = launch_scan_by_width<T, D, G, __nv_bfloat16>(a, st);
+      else return cudaErrorInvalidValue;  // the compact summary cache is for bf16 models
+    } else {
+      e = launch_scan_by_width<T, D, G, float>(a, st);
+    }
+    if (e != cudaSuccess) return e;
+  }
+  a.att_ctas = (2 * (a.top_k + 1) + kAttWarps - 1) / kAttWarps;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(bg * a.att_ctas);
+  cfg.blockDim = dim3(kAttWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = a.top_k > 0 ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_attend_kernel<T, D, G>, a);
+}
+
+}  // namespace hils
