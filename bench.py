@@ -89,57 +89,103 @@ def load_peaks():
 
 
 class Clocks:
-    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    """Samples the SM clock and the throttle reasons while running (read-only queries).
+
+    NVML is polled every ~2 ms from a thread, so that even a timed region of a few
+    milliseconds gets several samples; the device is found by its UUID, so the reading
+    is of this process's GPU whatever the visible-device mapping.  Without NVML it falls
+    back to `nvidia-smi -lms 100`.
+    """
 
     Q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    # NVML clocks-event reason bits, in the order of NAMES
+    BITS = (0x8, 0x40, 0x20, 0x4)
 
-    def __init__(self, index):
+    def __init__(self, index, period_s=0.002):
         self.index = index
+        self.period = period_s
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.stop = threading.Event()
+        self.samples = []  # (sm MHz, max sm MHz, frozenset of active reasons)
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            u = str(torch.cuda.get_device_properties(self.index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _nvml_sample(self, nv, h, mx):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.samples.append((float(sm), mx, frozenset(n for n, bit in zip(self.NAMES, self.BITS) if r & bit)))
+
+    def _nvml_loop(self, nv, h, mx):
+        while not self.stop.is_set():
+            try:
+                self._nvml_sample(nv, h, mx)
+            except Exception:
+                return
+            self.stop.wait(self.period)
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._nvml_sample(nv, h, mx)  # one reading before the timed work starts
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, mx), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.samples = []
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            active = frozenset(n for n, v in zip(self.NAMES, parts[2:6]) if v.lower().startswith("active"))
+            self.samples.append((sm, mx, active))
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 6:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[2:6]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
+        sm = [x[0] for x in self.samples]
+        mx = self.samples[-1][1] if self.samples else None
+        reasons = set().union(*[x[2] for x in self.samples]) if self.samples else set()
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def dist_setup(args=None, backend="nccl"):

@@ -67,3 +67,45 @@ def test_reference_arm_is_silent_off_rank_zero(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(Args())
     assert buf.getvalue() == ""
+
+
+class _FakeNvml:
+    """Stands in for the NVML binding: a fixed clock, power cap active on the 2nd reading."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self):
+        self.calls = 0
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return 1900
+
+    def nvmlDeviceGetCurrentClocksThrottleReasons(self, h):
+        self.calls += 1
+        return 0x4 if self.calls == 2 else 0
+
+
+def test_clock_sampler_polls_nvml_during_the_region(monkeypatch):
+    fake = _FakeNvml()
+    monkeypatch.setattr(bench.Clocks, "_nvml_handle", lambda self: (fake, object()))
+    with bench.Clocks(0, period_s=0.001) as clk:
+        import time
+        time.sleep(0.05)
+    s = clk.summary()
+    assert s["source"] == "nvml" and s["samples"] >= 3
+    assert s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_parses_nvidia_smi_lines():
+    clk = bench.Clocks(0)
+    clk.proc = type("P", (), {"stdout": io.StringIO(
+        "1965, 1965, Not Active, Not Active, Not Active, Not Active\n"
+        "1800, 1965, Not Active, Active, Not Active, Active\n"
+        "garbage\n")})()
+    clk._read()
+    s = clk.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1882.5 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
