@@ -34,6 +34,22 @@ reason in the design notes of this repository):
 * Scale 1/sqrt(d) everywhere unless a scale is given.
 * 0 * log 0 = 0 in the entropy.
 
+* Sliding-window local branch (notes section 5.2: the main configuration
+  keeps a 512-token sliding window next to the remote chunks; section 5.3:
+  the window's exact mass enters the normaliser Zhat_i beside the selected
+  chunks' surrogate masses).  With window W (a multiple of B) the local branch
+  is chunk-aligned: the own partial chunk and the W/B - 1 complete chunks
+  before it, keys [max(0, (c_i + 1 - W/B) * B), i], at their exact mass; the
+  remote candidates are the complete chunks before that, c < c_i + 1 - W/B.
+  W = B (the default) is the own-chunk branch above.
+* The row normaliser log Zhat_i (returned as "lse") is the log-sum-exp of the
+  fusion logits: the selected chunks' shat and the local branch's LSE.
+* Gradients (notes section 5.3: the hierarchical softmax lets the LM loss
+  train the selector; Tide Figure 3 caption: gradients reach the compressed
+  key): the Top-K indices are a constant of the backward pass; every other
+  step (intra-chunk softmax, inter-chunk softmax, shat = q.kbar*scale + H,
+  the landmark softmax that makes kbar and H) is differentiated exactly.
+
 Modes: "landmark" (the method), "exact" (shat replaced by the exact chunk
 log-mass log Z_{i,c}, notes section 3: naive block-sparse attention), and
 forced selection (the caller supplies I_i).
@@ -55,6 +71,8 @@ __all__ = [
     "forward",
     "decode",
     "summarize_pages",
+    "backward",
+    "summarize_backward",
 ]
 
 
@@ -66,6 +84,25 @@ def _f64(x):
 
 def _scale(d, scale):
     return 1.0 / math.sqrt(d) if (scale is None or scale == 0) else float(scale)
+
+
+def _local_chunks(chunk, window):
+    """Chunks in the local branch: 1 (own chunk only) or W / B for a window W."""
+    if window is None or window == 0:
+        return 1
+    if window % chunk != 0 or window < chunk:
+        raise ValueError("window must be a positive multiple of the chunk size")
+    return window // chunk
+
+
+def _n_cand(rows, chunk, window):
+    """Number of remote candidate chunks of each query position: c < c_i + 1 - W/B."""
+    return np.maximum(np.asarray(rows) // chunk + 1 - _local_chunks(chunk, window), 0)
+
+
+def _local_start(i, chunk, window):
+    """First key of query i's local branch."""
+    return max(0, (i // chunk + 1 - _local_chunks(chunk, window)) * chunk)
 
 
 # ---------------------------------------------------------------------------
@@ -114,8 +151,9 @@ def summarize(k, landmark, chunk, scale=None):
 # ---------------------------------------------------------------------------
 # 2. Chunk scores (notes section 5.2) and the exact chunk log-mass (section 3)
 # ---------------------------------------------------------------------------
-def chunk_scores(q, kbar, hbias, chunk, scale=None, rows=None):
-    """shat [b, h, R, C]: q_i . kbar_c * scale + H_c, -inf where c >= floor(i/B).
+def chunk_scores(q, kbar, hbias, chunk, scale=None, rows=None, window=None):
+    """shat [b, h, R, C]: q_i . kbar_c * scale + H_c, -inf where c is not a
+    remote candidate (c >= floor(i/B), or inside the local window).
 
     rows: query positions to score (default: all).
     """
@@ -127,14 +165,15 @@ def chunk_scores(q, kbar, hbias, chunk, scale=None, rows=None):
     rows = np.arange(n) if rows is None else np.asarray(rows)
     c_all = kbar.shape[2]
     s = np.einsum("bhrd,bhcd->bhrc", q[:, :, rows], kbar) * sc + hbias[:, :, None, :]
-    cand = np.arange(c_all)[None, :] < (rows // chunk)[:, None]
+    cand = np.arange(c_all)[None, :] < _n_cand(rows, chunk, window)[:, None]
     return np.where(cand[None, None], s, -np.inf)
 
 
-def exact_chunk_lse(q, k, chunk, scale=None, rows=None):
+def exact_chunk_lse(q, k, chunk, scale=None, rows=None, window=None):
     """log Z_{i,c} = log sum_{j in chunk c} exp(q_i . k_j * scale) (notes section 3).
 
-    Returned for complete chunks c < floor(i/B); -inf elsewhere.  [b, h, R, C]
+    Returned for the remote candidates c < floor(i/B) + 1 - W/B; -inf
+    elsewhere.  [b, h, R, C]
     """
     q = _f64(q)
     k = _f64(k)
@@ -151,7 +190,7 @@ def exact_chunk_lse(q, k, chunk, scale=None, rows=None):
             lg = np.einsum("rd,cjd->rcj", q[bi, hi, rows], kc[bi, hi // grp]) * sc
             m = lg.max(axis=2, keepdims=True)
             lse = np.log(np.exp(lg - m).sum(axis=2)) + m[..., 0]
-            cand = np.arange(c_all)[None, :] < (rows // chunk)[:, None]
+            cand = np.arange(c_all)[None, :] < _n_cand(rows, chunk, window)[:, None]
             out[bi, hi] = np.where(cand, lse, -np.inf)
     return out
 
@@ -196,7 +235,8 @@ def _softmax_attend(qv, keys, vals, sc):
 
 
 def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
-            forced_idx=None, rows=None, heads=None, q_score=None):
+            forced_idx=None, rows=None, heads=None, q_score=None, window=None,
+            keep_terms=False):
     """HiLS forward for a contiguous causal sequence.
 
     q [b,h,N,d], k/v [b,g,N,d], landmark [b,h,C,d] (C = N // chunk).
@@ -206,11 +246,15 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
     whole GQA group).  q_score [b,h,N,d]: a separate scoring query (notes
     section 5.4, the Q-Cal interface): it replaces q in the chunk scores, so it
     decides the selection and the inter-chunk weights, while q keeps the
-    intra-chunk attention and the own chunk.
+    intra-chunk attention and the local branch.  window: None (own chunk) or
+    a multiple W of the chunk size (sliding-window local branch).
 
     Returns a dict with out [b,h,R,d] (nan for heads not produced),
     idx [b,g,R,K], shat_sel [b,h,R,K] (-inf in unused slots), lse_own
-    [b,h,R], key [b,g,R,C] and shat [b,h,R,C].
+    [b,h,R] (log-mass of the local branch), lse [b,h,R] (log Zhat_i, the
+    log-sum-exp of all fusion logits), key [b,g,R,C] and shat [b,h,R,C].
+    With keep_terms, "terms" maps (b, h, t) to the per-branch pieces the
+    backward pass reuses.
     """
     q64, k64, v64 = _f64(q), _f64(k), _f64(v)
     b, h, n, d = q64.shape
@@ -221,9 +265,9 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
     qs64 = q64 if q_score is None else _f64(q_score)
     if mode == "landmark":
         kbar, hb = summarize(k64, landmark, chunk, scale)
-        shat = chunk_scores(qs64, kbar, hb, chunk, scale, rows)
+        shat = chunk_scores(qs64, kbar, hb, chunk, scale, rows, window)
     elif mode == "exact":
-        shat = exact_chunk_lse(qs64, k64, chunk, scale, rows)
+        shat = exact_chunk_lse(qs64, k64, chunk, scale, rows, window)
     else:
         raise ValueError(mode)
     if forced_idx is None:
@@ -236,6 +280,8 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
     out = np.full((b, h, r, d), np.nan)
     shat_sel = np.full((b, h, r, kk), -np.inf)
     lse_own = np.full((b, h, r), np.nan)
+    lse = np.full((b, h, r), np.nan)
+    terms_kept = {}
     want = set(heads) if heads is not None else None
     for bi in range(b):
         for hi in range(h):
@@ -245,11 +291,10 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
             for t, i in enumerate(rows):
                 i = int(i)
                 qv = q64[bi, hi, i]
-                own = i // chunk
-                o_own, l_own = _softmax_attend(qv, k64[bi, gi, own * chunk: i + 1],
-                                               v64[bi, gi, own * chunk: i + 1], sc)
+                lo = _local_start(i, chunk, window)
+                o_own, l_own = _softmax_attend(qv, k64[bi, gi, lo: i + 1], v64[bi, gi, lo: i + 1], sc)
                 lse_own[bi, hi, t] = l_own
-                terms = [(l_own, o_own)]
+                terms = [(l_own, o_own, -1)]
                 for s_, c in enumerate(idx[bi, gi, t]):
                     if c < 0:
                         continue
@@ -258,12 +303,142 @@ def forward(q, k, v, landmark, chunk, top_k, scale=None, mode="landmark",
                                              v64[bi, gi, c * chunk:(c + 1) * chunk], sc)
                     sh = shat[bi, hi, t, c]
                     shat_sel[bi, hi, t, s_] = sh
-                    terms.append((sh, o_c))
-                mx = max(x for x, _ in terms)
-                w = np.array([math.exp(x - mx) for x, _ in terms])
-                w /= w.sum()
-                out[bi, hi, t] = sum(wi * o for wi, (_, o) in zip(w, terms))
-    return dict(out=out, idx=idx, shat_sel=shat_sel, lse_own=lse_own, key=key, shat=shat)
+                    terms.append((sh, o_c, c))
+                mx = max(x for x, _, _ in terms)
+                w = np.array([math.exp(x - mx) for x, _, _ in terms])
+                z = w.sum()
+                w /= z
+                lse[bi, hi, t] = mx + math.log(z)
+                out[bi, hi, t] = sum(wi * o for wi, (_, o, _) in zip(w, terms))
+                if keep_terms:
+                    terms_kept[bi, hi, t] = (lo, w, terms)
+    res = dict(out=out, idx=idx, shat_sel=shat_sel, lse_own=lse_own, lse=lse, key=key, shat=shat)
+    if keep_terms:
+        res["terms"] = terms_kept
+    return res
+
+
+# ---------------------------------------------------------------------------
+# 4b. Backward pass (notes section 5.3; Tide Figure 3 caption)
+# ---------------------------------------------------------------------------
+def summarize_backward(keys, landmark, scale, dkbar, dh):
+    """Chain rule through one chunk summary (notes section 5.1).
+
+    sigma_j = l . k_j * scale, pi = softmax(sigma), kbar = sum_j pi_j k_j,
+    H = -sum_j pi_j log pi_j.  Given dL/dkbar [d] and dL/dH, returns
+    dL/dkeys [B, d] and dL/dl [d]:
+      dpi_j    = dkbar . k_j - dH (log pi_j + 1)
+      dsigma_j = pi_j (dpi_j - sum_m pi_m dpi_m)
+      dk_j     = pi_j dkbar + scale dsigma_j l,   dl = scale sum_j dsigma_j k_j.
+    log pi_j is taken as sigma_j - LSE(sigma), finite even where pi_j
+    underflows to 0 (there pi_j multiplies it, so 0 log 0 = 0 still holds).
+    """
+    sig = keys @ landmark * scale
+    m = sig.max()
+    e = np.exp(sig - m)
+    z = e.sum()
+    pi = e / z
+    logpi = sig - (m + math.log(z))
+    dpi = keys @ dkbar - dh * (logpi + 1.0)
+    dsig = pi * (dpi - pi @ dpi)
+    dkeys = pi[:, None] * dkbar[None, :] + scale * dsig[:, None] * landmark[None, :]
+    dl = scale * (dsig @ keys)
+    return dkeys, dl
+
+
+def backward(q, k, v, landmark, dout, chunk, top_k, scale=None, mode="landmark",
+             forced_idx=None, rows=None, heads=None, q_score=None, window=None):
+    """Gradients of L = sum(dout * out) for the HiLS forward pass.
+
+    Arguments as for forward(); dout has out's shape [b,h,R,d] for the rows
+    given (default all).  The selection I_i is held fixed (Top-K is not
+    differentiable); everything else is differentiated exactly.  Only the
+    listed rows and (b, h) pairs contribute, so a caller can assemble the
+    gradient of a key from the rows that attend to it.
+
+    Per row i with fusion weights w (local branch l, selected chunks c),
+    output o and D = dout . o:
+      selected chunk c:  dshat_c = w_c (dout . o_c - D)
+                         ds_ij   = w_c p_ij (dout . v_j - dout . o_c)
+      local branch:      ds_ij   = w_l p_ij (dout . v_j - D)
+                         (its logit is LSE_l, whose gradient is p_ij)
+      every key j used:  dv_j += w p_ij dout,  dk_j += scale ds_ij q_i,
+                         dq_i += scale ds_ij k_j
+      scores:            dq_i (or dq_score_i) += scale dshat_c kbar_c,
+                         dkbar_c += scale dshat_c q_i (q_score_i), dH_c += dshat_c
+    then summarize_backward() carries dkbar, dH to the chunk keys and the
+    landmark query.  In "exact" mode the chunk logit is LSE_c, so its
+    keys get ds_ij = w_c p_ij (dout . v_j - D) and no summary gradient.
+
+    Returns dict dq [b,h,N,d], dk, dv [b,g,N,d], dlandmark [b,h,C,d],
+    dq_score [b,h,N,d] (None without q_score), dkbar [b,h,C,d], dhbias [b,h,C].
+    """
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    lm64 = _f64(landmark)
+    b, h, n, d = q64.shape
+    g = k64.shape[1]
+    grp = h // g
+    sc = _scale(d, scale)
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    do = _f64(dout)
+    qs64 = q64 if q_score is None else _f64(q_score)
+    fw = forward(q64, k64, v64, lm64, chunk, top_k, scale, mode, forced_idx, rows, heads,
+                 q_score=q_score, window=window, keep_terms=True)
+    c_all = n // chunk
+    dq = np.zeros_like(q64)
+    dqs = np.zeros_like(q64)
+    dk = np.zeros_like(k64)
+    dv = np.zeros_like(v64)
+    dkbar = np.zeros((b, h, c_all, d))
+    dhb = np.zeros((b, h, c_all))
+    kbar = None
+    if mode == "landmark":
+        kbar, _ = summarize(k64, lm64, chunk, scale)
+    for (bi, hi, t), (lo, w, terms) in fw["terms"].items():
+        gi = hi // grp
+        i = int(rows[t])
+        qv = q64[bi, hi, i]
+        g_o = do[bi, hi, t]
+        o = fw["out"][bi, hi, t]
+        D = g_o @ o
+        for wx, (_, o_x, c) in zip(w, terms):
+            if c < 0:
+                j0, j1 = lo, i + 1
+            else:
+                j0, j1 = c * chunk, (c + 1) * chunk
+            keys, vals = k64[bi, gi, j0:j1], v64[bi, gi, j0:j1]
+            lg = keys @ qv * sc
+            p = np.exp(lg - lg.max())
+            p /= p.sum()
+            dov = vals @ g_o
+            if c < 0 or mode == "exact":
+                ds = wx * p * (dov - D)
+            else:
+                ds = wx * p * (dov - g_o @ o_x)
+                dsh = wx * (g_o @ o_x - D)
+                dqs[bi, hi, i] += sc * dsh * kbar[bi, hi, c]
+                dkbar[bi, hi, c] += sc * dsh * qs64[bi, hi, i]
+                dhb[bi, hi, c] += dsh
+            dv[bi, gi, j0:j1] += (wx * p)[:, None] * g_o[None, :]
+            dk[bi, gi, j0:j1] += sc * ds[:, None] * qv[None, :]
+            dq[bi, hi, i] += sc * (ds @ keys)
+    dlm = np.zeros_like(lm64)
+    if mode == "landmark":
+        for bi in range(b):
+            for hi in range(h):
+                gi = hi // grp
+                for c in range(c_all):
+                    if dhb[bi, hi, c] == 0.0 and not dkbar[bi, hi, c].any():
+                        continue
+                    sl = slice(c * chunk, (c + 1) * chunk)
+                    dkeys, dl = summarize_backward(k64[bi, gi, sl], lm64[bi, hi, c], sc,
+                                                   dkbar[bi, hi, c], dhb[bi, hi, c])
+                    dk[bi, gi, sl] += dkeys
+                    dlm[bi, hi, c] = dl
+    if q_score is None:
+        dq += dqs
+        dqs = None
+    return dict(dq=dq, dk=dk, dv=dv, dlandmark=dlm, dq_score=dqs, dkbar=dkbar, dhbias=dhb)
 
 
 # ---------------------------------------------------------------------------
@@ -289,16 +464,18 @@ def summarize_pages(k_pages, landmark_pages, page_ids, heads_q, scale=None):
 
 
 def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
-           scale=None, batches=None):
+           scale=None, batches=None, window=None):
     """One decode step per sequence.
 
     q [b,h,d] is the query at position seq_lens[b]-1, whose key/value are
     already in the cache.  Chunk c of sequence b lives in page
     block_table[b, c] of the pools k_pages/v_pages [P,g,B,d].  The own chunk is
-    floor((seq_len-1)/B); candidates are the complete chunks before it, scored
+    floor((seq_len-1)/B); candidates are the complete chunks before the local
+    branch (the own chunk, or with a window W the last W/B chunks), scored
     with summaries computed here from landmark_pages [P,h,d].
-    Returns out [b,h,d] (zeros for seq_len <= 0), idx [b,g,K] and, per
-    sequence, the selection key [g, own] of its candidate chunks.
+    Returns out [b,h,d] (zeros for seq_len <= 0), idx [b,g,K], lse [b,h]
+    (log Zhat) and, per sequence, the selection key [g, n_cand] of its
+    candidate chunks.
     """
     q64, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
     bt = np.asarray(block_table).astype(np.int64)
@@ -311,27 +488,31 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
     out = np.zeros((b, h, d))
     idx = np.full((b, g, top_k), -1, dtype=np.int64)
     shat_sel = np.full((b, h, top_k), -np.inf)
+    lse = np.full((b, h), -np.inf)
     keys = {}
     for bi in range(b) if batches is None else batches:
         L = int(sl[bi])
         if L <= 0:
             continue
         own = (L - 1) // chunk
-        pages = bt[bi, :own]
+        n_cand = int(_n_cand(L - 1, chunk, window))
+        pages = bt[bi, :n_cand]
         summ = summarize_pages(kp, landmark_pages, pages, h, scale)
-        shat = np.full((h, own), -np.inf)
-        for c in range(own):
+        shat = np.full((h, n_cand), -np.inf)
+        for c in range(n_cand):
             kb, hb = summ[int(pages[c])]
             shat[:, c] = np.einsum("hd,hd->h", kb, q64[bi]) * sc + hb
         sel, key = select_topk(shat[None, :, None, :], g, top_k)
         idx[bi] = sel[0, :, 0]
         keys[bi] = key[0, :, 0]
-        own_page = int(bt[bi, own])
-        n_own = L - own * chunk
+        lo_c = _local_start(L - 1, chunk, window) // chunk
         for hi in range(h):
             gi = hi // grp
             qv = q64[bi, hi]
-            o_own, l_own = _softmax_attend(qv, kp[own_page, gi, :n_own], vp[own_page, gi, :n_own], sc)
+            # local branch: chunks lo_c .. own, the last one up to the new token
+            lk = np.concatenate([kp[int(bt[bi, c]), gi, :min(chunk, L - c * chunk)] for c in range(lo_c, own + 1)])
+            lv = np.concatenate([vp[int(bt[bi, c]), gi, :min(chunk, L - c * chunk)] for c in range(lo_c, own + 1)])
+            o_own, l_own = _softmax_attend(qv, lk, lv, sc)
             terms = [(l_own, o_own)]
             for s_, c in enumerate(idx[bi, gi]):
                 if c < 0:
@@ -342,6 +523,8 @@ def decode(q, k_pages, v_pages, landmark_pages, block_table, seq_lens, top_k,
                 shat_sel[bi, hi, s_] = shat[hi, int(c)]
             mx = max(x for x, _ in terms)
             w = np.array([math.exp(x - mx) for x, _ in terms])
-            w /= w.sum()
+            z = w.sum()
+            w /= z
+            lse[bi, hi] = mx + math.log(z)
             out[bi, hi] = sum(wi * o for wi, (_, o) in zip(w, terms))
-    return dict(out=out, idx=idx, shat_sel=shat_sel, key=keys)
+    return dict(out=out, idx=idx, shat_sel=shat_sel, key=keys, lse=lse)
