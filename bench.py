@@ -147,8 +147,14 @@ class Clocks:
         except Exception:
             self.samples = []
         try:
+            # nvidia-smi numbers GPUs without regard to CUDA_VISIBLE_DEVICES: address the device by UUID
+            try:
+                u = str(torch.cuda.get_device_properties(self.index).uuid)
+                dev_id = u if u.startswith("GPU-") else "GPU-" + u
+            except Exception:
+                dev_id = str(self.index)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", "-i", dev_id, f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.source = "nvidia-smi"
             self.thread = threading.Thread(target=self._read, daemon=True)
@@ -227,36 +233,100 @@ def job_tflops(ws, flops_per_replica, ms_max):
 
 
 # ---------------------------------------------------------------------------- CPU baseline (oracle)
-def cpu_baseline(seconds_budget=20.0):
-    """Times the fp64 oracle on a bounded sample of the prefill workload."""
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds_budget=20.0, threads=None, cfg_name="prefill_345m", inp=None, row_stride=1):
+    """Times the fp64 oracle, as it stands, on a bounded sample of a prefill workload:
+    (batch, KV group) slices, in order, until the time budget is spent, each with every
+    row_stride-th query row.  The throughput is the algorithmic FLOPs of the rows done
+    over the time taken.  threads: BLAS threads (None = every host core)."""
     from threadpoolctl import threadpool_limits
 
     from oracle import hils_oracle as O
-    cfg = dict(PREFILL)
-    inp = prefill_inputs(seed=0, device="cpu", **cfg)
-    n = cfg["seq_len"]
-    # sample: whole (batch, head) pairs in order until the time budget is spent
-    t0 = time.perf_counter()
-    flops, done_rows, pairs = 0.0, 0, 0
-    rows = np.arange(n)
+    cfg = dict(CONFIGS[cfg_name])
+    if inp is None:
+        inp = prefill_inputs(seed=0, device="cpu", **cfg)
+    n, grp = cfg["seq_len"], cfg["heads_q"] // cfg["heads_kv"]
+    rows = np.arange(0, n, row_stride)
     keff = np.minimum(cfg["top_k"], rows // 64)
-    pair_flops = float(4 * cfg["head_dim"] * (keff * 64 + rows % 64 + 1).sum())
-    with threadpool_limits(limits=1):
+    head_flops = float(4 * cfg["head_dim"] * (keff * 64 + rows % 64 + 1).sum())
+    full_flops = algorithmic_flops(cfg["batch"], cfg["heads_q"], n, cfg["head_dim"], cfg["top_k"])
+    cores = threads or host_cores()
+    t0 = time.perf_counter()
+    flops, slices = 0.0, 0
+    with threadpool_limits(limits=cores):
         for bi in range(cfg["batch"]):
-            for hi in range(cfg["heads_q"]):
-                if time.perf_counter() - t0 >= seconds_budget:
+            for gi in range(cfg["heads_kv"]):
+                if slices and time.perf_counter() - t0 >= seconds_budget:
                     break
-                O.forward(inp.q[bi:bi + 1, hi:hi + 1], inp.k[bi:bi + 1, hi:hi + 1],
-                          inp.v[bi:bi + 1, hi:hi + 1], inp.landmark[bi:bi + 1, hi:hi + 1], 64,
-                          cfg["top_k"])
-                flops += pair_flops
-                pairs += 1
+                hs = slice(gi * grp, (gi + 1) * grp)
+                O.forward(inp.q[bi:bi + 1, hs], inp.k[bi:bi + 1, gi:gi + 1], inp.v[bi:bi + 1, gi:gi + 1],
+                          inp.landmark[bi:bi + 1, hs], 64, cfg["top_k"], rows=None if row_stride == 1 else rows)
+                flops += head_flops * grp
+                slices += 1
     dt = time.perf_counter() - t0
-    done = pairs * n
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-            "sample": f"{pairs} of {cfg['batch'] * cfg['heads_q']} (batch, head) pairs, all {n} query rows "
-                      f"each (summaries, scores, Top-K, attention, fusion), {dt:.1f} s, fp64 numpy, "
-                      f"BLAS limited to 1 thread"}
+    total = cfg["batch"] * cfg["heads_kv"]
+    rows_txt = f"all {n} query rows" if row_stride == 1 else f"every {row_stride}th of {n} query rows"
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds": round(dt, 2), "full_config_seconds_scaled": round(dt * full_flops / flops, 1),
+            "sample": f"{cfg_name}: {slices} of {total} (batch, KV group) slices, {rows_txt} each "
+                      f"(summaries, scores, Top-K, attention, fusion), {dt:.1f} s, fp64 numpy, "
+                      f"BLAS on {cores} thread(s); full-config time scaled by algorithmic FLOPs"}
+
+
+def cpu_decode_baseline(name, seconds_budget=10.0, threads=None):
+    """The oracle's decode step on whole (sequence, KV head) slices of a decode workload
+    (each slice drawn on its own, with the workload's shape), scaled by slice count to
+    the whole batch (tokens/s)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import hils_oracle as O
+    cfg = dict(CONFIGS[name])
+    grp = cfg["heads_q"] // cfg["heads_kv"]
+    cores = threads or host_cores()
+    spent, slices = 0.0, 0
+    while slices == 0 or spent < seconds_budget:
+        one = dict(cfg, batch=1, heads_q=grp, heads_kv=1)
+        di = decode_inputs(seed=slices, device="cpu", **one)
+        t0 = time.perf_counter()
+        with threadpool_limits(limits=cores):
+            O.decode(di.q, di.k_pages, di.v_pages, di.landmark_pages, di.block_table.numpy(),
+                     di.seq_lens.numpy(), cfg["top_k"])
+        spent += time.perf_counter() - t0
+        slices += 1
+        if slices >= cfg["batch"] * cfg["heads_kv"]:
+            break
+    total = cfg["batch"] * cfg["heads_kv"]
+    step_s = spent * total / slices
+    return {"tok_s": cfg["batch"] / step_s, "seconds": round(spent, 2), "full_step_seconds_scaled": round(step_s, 2),
+            "cores": cores, "kind": "oracle",
+            "sample": f"{name}: {slices} of {total} (sequence, KV head) slices of one decode step, each drawn "
+                      f"alone with the workload's shape, scaled by slice count"}
+
+
+def oracle_times(budget):
+    """Oracle seconds beside the GPU time for every workload (each a bounded, stated sample)."""
+    res = {}
+    from threadpoolctl import threadpool_limits
+
+    from oracle import hils_oracle as O
+    cfg = CONFIGS["tiny_fp32"]
+    inp = prefill_inputs(seed=0, device="cpu", **cfg)
+    for cores in (1, None):
+        t0 = time.perf_counter()
+        with threadpool_limits(limits=cores or host_cores()):
+            O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, cfg["top_k"])
+        res["tiny_fp32" + ("_1core" if cores == 1 else "")] = {
+            "seconds": round(time.perf_counter() - t0, 3), "cores": cores or host_cores(), "sample": "full config"}
+    res["prefill_7b_gqa"] = cpu_baseline(budget, cfg_name="prefill_7b_gqa", row_stride=16)
+    for name in ("decode_32k", "decode_128k", "decode_512k"):
+        res[name] = cpu_decode_baseline(name, budget / 2)
+    return res
 
 
 # ---------------------------------------------------------------------------- prefill (ours)
@@ -293,7 +363,7 @@ def run_prefill(args, ws_world, rank, local):
         if evs: evs[1].record(stream)
         r |= lib.hils_select(ctypes.byref(sh), P(q), P(kb), P(hbb), P(idx), P(ssel), P(ws_sel), ws_sel.numel(), st)
         if evs: evs[2].record(stream)
-        r |= lib.hils_attend_selected(ctypes.byref(sh), P(q), P(k), P(v), P(idx), P(ssel), P(out),
+        r |= lib.hils_attend_selected(ctypes.byref(sh), P(q), P(k), P(v), P(idx), P(ssel), P(out), None,
                                       P(ws_sel), ws_sel.numel(), st)
         if evs: evs[3].record(stream)
         if r != 0:
@@ -312,8 +382,9 @@ def run_prefill(args, ws_world, rank, local):
     att = [e[2].elapsed_time(e[3]) for e in evsets]
     summ = [e[0].elapsed_time(e[1]) for e in evsets]
     sel = [e[1].elapsed_time(e[2]) for e in evsets]
-    ms_step = max_over_ranks(sum(tot) / len(tot), ws_world)
-    ms_att = sum(att) / len(att)
+    ms_step = max_over_ranks(statistics.median(tot), ws_world)
+    ms_att = statistics.median(att)
+    recall = needle_recall(inp.needles, idx, h // g)
 
     # End to end through the public API with host buffers (pinned): every step uploads its
     # inputs and downloads its output inside the timed region.  Two buffer sets and three
@@ -352,7 +423,7 @@ def run_prefill(args, ws_world, rank, local):
     e2e_steps(max(2, args.warmup))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(4, args.steps // 2)
+    n_e2e = args.steps
     e0.record(up)  # before the first upload
     e2e_steps(n_e2e)
     e1.record(down)  # after the last download, which follows every other step's work
@@ -361,9 +432,20 @@ def run_prefill(args, ws_world, rank, local):
     assert call.device_status() == 0
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = host_out[0].numel() * host_out[0].element_size()
-    return dict(flops=flops, ms_step=ms_step, ms_att=ms_att, ms_summ=sum(summ) / len(summ),
-                ms_sel=sum(sel) / len(sel), ms_e2e=ms_e2e, h2d=h2d, d2h=d2h, clocks=clk.summary(),
-                launches_per_step=3)
+    return dict(flops=flops, ms_step=ms_step, ms_att=ms_att, ms_summ=statistics.median(summ),
+                ms_sel=statistics.median(sel), ms_e2e=ms_e2e, h2d=h2d, d2h=d2h, clocks=clk.summary(),
+                launches_per_step=3, needle_recall=recall)
+
+
+def needle_recall(needles, idx, group):
+    """Diagnostic (not parity): the fraction of planted needles (b, h, c, j, i) whose
+    target query i selected the needle's chunk c."""
+    if not needles:
+        return None
+    t = torch.tensor([[b, h // group, i, c] for b, h, c, j, i in needles], device=idx.device)
+    sel = idx[t[:, 0], t[:, 1], t[:, 2]]
+    hit = (sel == t[:, 3:4]).any(dim=1)
+    return {"hits": int(hit.sum()), "needles": len(needles), "fraction": round(float(hit.float().mean()), 4)}
 
 
 def run_prefill_gqa(dev, steps=5, warmup=3):
@@ -394,7 +476,7 @@ def run_prefill_gqa(dev, steps=5, warmup=3):
     med = [statistics.median(t[i] for t in times) for i in range(3)]
     flops = algorithmic_flops(b, h, n, d, K)
     return {"workload": "prefill_7b_gqa: batch 1, 32 query heads / 8 KV heads, N 32768, d 128, top-k 32, bf16",
-            "ms_per_step": round(sum(med), 4),
+            "ms_per_step": round(sum(med), 4), "needle_recall": needle_recall(inp.needles, idx, h // g),
             "stage_ms": {"summarize": round(med[0], 4), "select": round(med[1], 4), "attend_selected": round(med[2], 4)},
             "tflops": round(flops / (sum(med) * 1e-3) / 1e12, 3),
             "attend_tflops": round(flops / (med[2] * 1e-3) / 1e12, 3),
@@ -441,19 +523,19 @@ def run_decode(name, n_caches, dev, reps=50):
         for gr in graphs:
             gr.replay()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record()
         for r in range(reps):
             graphs[r % len(graphs)].replay()
-        e1.record()
+            evs[r + 1].record()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / reps
+        ms = statistics.median(evs[r].elapsed_time(evs[r + 1]) for r in range(reps))
         for (di, kbars, call, out) in caches:
             assert call.device_status() == 0
         alg, kv_only = decode_bytes(cfg, sbytes)
         del graphs
         res[dt] = dict(ms=ms, tok_s=cfg["batch"] / (ms * 1e-3), gbs=alg / (ms * 1e-3) / 1e9, bytes=alg,
-                       kv_bytes=kv_only)
+                       kv_bytes=kv_only, caches=n_caches, reps=reps)
     del caches
     torch.cuda.empty_cache()
     return res
@@ -466,8 +548,8 @@ def run_ours(args):
     dec = {}
     if not args.no_decode:
         for name in args.decode_configs.split(","):
-            nc = 3 if name == "decode_32k" else 1   # 3 rotating caches keep 32K out of L2
-            r = run_decode(name, nc, torch.device("cuda", local))
+            # three rotating caches (each larger than L2 from 128K up) keep every step's reads in HBM
+            r = run_decode(name, 3, torch.device("cuda", local))
             dec[name] = r[torch.float32]
             dec[name + "_bf16_summaries"] = r[torch.bfloat16]
     if args.decode_only:
@@ -478,7 +560,11 @@ def run_ours(args):
         return
     pre = run_prefill(args, ws_world, rank, local)
     gqa = run_prefill_gqa(torch.device("cuda", local)) if not args.no_gqa else None
-    cpu = cpu_baseline(args.cpu_seconds) if (rank == 0 and ws_world == 1 and not args.no_cpu) else None
+    cpu = cpu1 = otimes = None
+    if rank == 0 and ws_world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.cpu_seconds)                 # every host core
+        cpu1 = cpu_baseline(args.cpu_seconds / 2, threads=1)  # one core
+        otimes = oracle_times(args.cpu_seconds / 2)
     if ws_world > 1:
         torch.distributed.barrier()
     if rank != 0:
@@ -519,6 +605,8 @@ def run_ours(args):
                           "consecutive steps"},
         "gpu_launches": pre["launches_per_step"] * args.steps,
         "clocks": pre["clocks"],
+        "needle_recall": pre["needle_recall"],
+        "timing": "CUDA-event median over the timed steps",
     }
     if gqa:
         line["prefill_7b_gqa"] = gqa
@@ -527,10 +615,13 @@ def run_ours(args):
             k: {"tok_s": round(r["tok_s"], 1), "us_per_step": round(r["ms"] * 1e3, 2),
                 "alg_bytes": int(r["bytes"]), "kv_bytes": int(r["kv_bytes"]),
                 "achieved_gbs": round(r["gbs"], 1), "frac_hbm": round(r["gbs"] / hbm, 4),
-                "timing": "CUDA-graph replay, 2 kernels per step"}
+                "timing": f"CUDA-graph replay, 2 kernels per step, median of {r['reps']} steps rotating over "
+                          f"{r['caches']} independent caches"}
             for k, r in dec.items()}
     if cpu:
         line["cpu_baseline"] = cpu
+        line["cpu_baseline_1core"] = cpu1
+        line["oracle_times"] = otimes
     print(json.dumps(line), flush=True)
     if ws_world > 1:
         torch.distributed.destroy_process_group()
@@ -551,13 +642,16 @@ def run_reference(args):
                               PREFILL["top_k"])
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": flops / (value * 1e12) * 1e3,
+        "steps": args.steps, "warmup": args.warmup,
+        # each timed step is a bounded sample of the workload (see cpu_baseline.sample)
+        "ms_per_step": round(statistics.median(v["seconds"] for v in vals) * 1e3, 1),
+        "ms_per_full_step_extrapolated": round(flops / (value * 1e12) * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": "prefill_345m: batch 4, 16 heads (MHA), N 8192, d 64, chunk 64, top-k 16",
                    "global_batch": PREFILL["batch"], "seq_len": PREFILL["seq_len"], "parallelism": "cpu oracle"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": vals[-1]["sample"]},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": vals[-1]["cores"], "kind": "oracle",
+                         "sample": "each step: " + vals[-1]["sample"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -37,6 +37,7 @@ class Shape(ctypes.Structure):
         ("batch", ctypes.c_int32), ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("chunk", ctypes.c_int32),
         ("top_k", ctypes.c_int32), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+        ("window", ctypes.c_int32),
     ]
 
 
@@ -62,8 +63,8 @@ def lib():
         "hils_summarize": (i32, [S, _P, _P, _P, _P, _P]),
         "hils_summarize_paged": (i32, [S, _P, _P, _P, i32, i32, _P, _P, _P]),
         "hils_select": (i32, [S, _P, _P, _P, _P, _P, _P, sz, _P]),
-        "hils_attend": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
-        "hils_attend_selected": (i32, [S, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "hils_attend": (i32, [S, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
+        "hils_attend_selected": (i32, [S, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "hils_decode": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
         "hils_summarize_paged_ex": (i32, [S, _P, _P, _P, i32, i32, _P, i32, _P, _P]),
         "hils_decode_ex": (i32, [S, _P, _P, _P, _P, i32, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
@@ -111,8 +112,9 @@ def _check(st: int, where: str):
         raise HilsError(st, where)
 
 
-def make_shape(batch, heads_q, heads_kv, head_dim, seq_len, top_k, dtype, chunk=64, scale=0.0):
-    return Shape(batch, heads_q, heads_kv, head_dim, seq_len, chunk, top_k, float(scale or 0.0), dtype)
+def make_shape(batch, heads_q, heads_kv, head_dim, seq_len, top_k, dtype, chunk=64, scale=0.0, window=0):
+    return Shape(batch, heads_q, heads_kv, head_dim, seq_len, chunk, top_k, float(scale or 0.0), dtype,
+                 int(window or 0))
 
 
 def workspace_size(shape: Shape, op: int) -> int:
@@ -155,10 +157,10 @@ def summarize_paged(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages, 
                                          _ptr(hbias_pages), _stream(stream)), "hils_summarize_paged_ex")
 
 
-def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True):
+def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True, window=0):
     """topk_idx [b,g,N,K] int32 and (optionally) topk_score [b,h,N,K] fp32."""
     b, h, n, d = q.shape
-    sh = make_shape(b, h, heads_kv, d, n, top_k, _dt(q), scale=scale or 0.0)
+    sh = make_shape(b, h, heads_kv, d, n, top_k, _dt(q), scale=scale or 0.0, window=window)
     idx = torch.empty((b, heads_kv, n, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, h, n, top_k), dtype=torch.float32, device=q.device) if with_scores else None
     ws = new_workspace(sh, OP_SELECT, q.device)
@@ -170,13 +172,14 @@ def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores
 class Prefill:
     """Reusable prefill call: holds the workspace for one shape."""
 
-    def __init__(self, batch, heads_q, heads_kv, seq_len, head_dim, top_k, dtype, scale=None, device="cuda"):
+    def __init__(self, batch, heads_q, heads_kv, seq_len, head_dim, top_k, dtype, scale=None, device="cuda",
+                 window=0):
         self.shape = make_shape(batch, heads_q, heads_kv, head_dim, seq_len, top_k,
                                 HILS_BF16 if dtype in (torch.bfloat16, "bf16") else HILS_F32,
-                                scale=scale or 0.0)
+                                scale=scale or 0.0, window=window)
         self.ws = new_workspace(self.shape, OP_ATTEND, device)
 
-    def __call__(self, q, k, v, landmark, out=None, topk_idx=None, stream=None):
+    def __call__(self, q, k, v, landmark, out=None, topk_idx=None, stream=None, lse=None):
         s = self.shape
         if q.shape != (s.batch, s.heads_q, s.seq_len, s.head_dim) or _dt(q) != s.dtype:
             raise ValueError("q does not match the prepared shape")
@@ -185,8 +188,13 @@ class Prefill:
                 raise TypeError("q, k, v and landmark must share a dtype")
         if out is None:
             out = torch.empty_like(q)
+        if lse is not None and (lse.dtype != torch.float32 or lse.shape != q.shape[:3]):
+            raise ValueError("lse must be fp32 [b, h, seq_len]")
+        if topk_idx is not None and (topk_idx.dtype != torch.int32 or
+                                     topk_idx.shape != (s.batch, s.heads_kv, s.seq_len, s.top_k)):
+            raise ValueError("topk_idx must be int32 [b, heads_kv, seq_len, top_k]")
         _check(lib().hils_attend(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(landmark), _ptr(out),
-                                 _ptr(topk_idx), _ptr(self.ws), self.ws.numel(), _stream(stream)),
+                                 _ptr(lse), _ptr(topk_idx), _ptr(self.ws), self.ws.numel(), _stream(stream)),
                "hils_attend")
         return out
 
@@ -194,40 +202,52 @@ class Prefill:
         return lib().hils_device_status(_ptr(self.ws), _stream(stream))
 
 
-def attend(q, k, v, landmark, top_k, scale=None, stream=None, return_idx=False, q_score=None):
-    """HiLS prefill forward; returns out (and topk_idx if asked).
+def attend(q, k, v, landmark, top_k, scale=None, stream=None, return_idx=False, q_score=None, window=0,
+           return_lse=False):
+    """HiLS prefill forward; returns out, then topk_idx and lse [b,h,N] (log Zhat)
+    when asked.
 
     q_score: a separate scoring query (the Q-Cal interface): summaries, then
-    hils_select with q_score, then hils_attend_selected with q."""
+    hils_select with q_score, then hils_attend_selected with q.  window: 0 (the
+    own-chunk local branch) or a multiple of 64 (a chunk-aligned sliding window)."""
     b, h, n, d = q.shape
     g = k.shape[1]
+    lse = torch.empty((b, h, n), dtype=torch.float32, device=q.device) if return_lse else None
     if q_score is not None:
         if q_score.shape != q.shape or q_score.dtype != q.dtype:
             raise ValueError("q_score must match q's shape and dtype")
         kbar, hb = summarize(k, landmark, scale=scale, stream=stream)
-        idx, sc = select(q_score, kbar, hb, top_k, g, scale=scale, stream=stream)
-        out = attend_selected(q, k, v, idx, sc, scale=scale, stream=stream)
-        return (out, idx) if return_idx else out
-    call = Prefill(b, h, g, n, d, top_k, q.dtype, scale=scale, device=q.device)
-    idx = torch.empty((b, g, n, top_k), dtype=torch.int32, device=q.device) if return_idx else None
-    out = call(q, k, v, landmark, topk_idx=idx, stream=stream)
-    return (out, idx) if return_idx else out
+        idx, sc = select(q_score, kbar, hb, top_k, g, scale=scale, stream=stream, window=window)
+        out = attend_selected(q, k, v, idx, sc, scale=scale, stream=stream, window=window, lse=lse)
+    else:
+        call = Prefill(b, h, g, n, d, top_k, q.dtype, scale=scale, device=q.device, window=window)
+        idx = torch.empty((b, g, n, top_k), dtype=torch.int32, device=q.device) if return_idx else None
+        out = call(q, k, v, landmark, topk_idx=idx, stream=stream, lse=lse)
+    res = (out,) + ((idx,) if return_idx else ()) + ((lse,) if return_lse else ())
+    return res if len(res) > 1 else out
 
 
-def attend_selected(q, k, v, topk_idx, topk_score, scale=None, out=None, ws=None, stream=None):
-    """Attention + fusion for a given selection (topk_idx [b,g,N,K], topk_score [b,h,N,K])."""
+def attend_selected(q, k, v, topk_idx, topk_score, scale=None, out=None, ws=None, stream=None, window=0,
+                    lse=None):
+    """Attention + fusion for a given selection (topk_idx [b,g,N,K], topk_score [b,h,N,K]);
+    lse, if given (fp32 [b,h,N]), receives log Zhat."""
     b, h, n, d = q.shape
     g = k.shape[1]
     K = topk_idx.shape[-1]
-    sh = make_shape(b, h, g, d, n, K, _dt(q), scale=scale or 0.0)
+    sh = make_shape(b, h, g, d, n, K, _dt(q), scale=scale or 0.0, window=window)
     if topk_idx.dtype != torch.int32 or topk_score.dtype != torch.float32:
         raise TypeError("topk_idx must be int32 and topk_score fp32")
+    if topk_idx.shape != (b, g, n, K) or topk_score.shape != (b, h, n, K):
+        raise ValueError("topk_idx must be [b, heads_kv, N, K] and topk_score [b, heads_q, N, K]")
+    if lse is not None and (lse.dtype != torch.float32 or lse.shape != (b, h, n)):
+        raise ValueError("lse must be fp32 [b, h, N]")
     if out is None:
         out = torch.empty_like(q)
     if ws is None:
         ws = new_workspace(sh, OP_ATTEND_SELECTED, q.device)
     _check(lib().hils_attend_selected(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx),
-                                      _ptr(topk_score), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+                                      _ptr(topk_score), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                      _stream(stream)),
            "hils_attend_selected")
     return out
 
@@ -287,6 +307,16 @@ def decode_static(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq
         raise TypeError("block_table and seq_lens must be int32")
     if status_word is not None and (status_word.dtype != torch.int32 or status_word.numel() < 1):
         raise TypeError("status_word must be an int32 device tensor")
+    # the entry point reads fp32 summaries only (it has no summary-dtype argument)
+    if kbar_pages.dtype != torch.float32 or hbias_pages.dtype != torch.float32:
+        raise TypeError("decode_static needs fp32 kbar_pages and hbias_pages (use decode() for a bf16 cache)")
+    if kbar_pages.shape != (k_pages.shape[0], h, d) or hbias_pages.shape != (k_pages.shape[0], h):
+        raise ValueError("kbar_pages must be [n_pages, heads_q, d] and hbias_pages [n_pages, heads_q]")
+    if topk_idx is not None and (topk_idx.dtype != torch.int32 or topk_idx.numel() < b * g * top_k):
+        raise TypeError("topk_idx must be an int32 tensor of at least batch * heads_kv * top_k entries")
+    for t in (q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, topk_idx, status_word, out):
+        if t is not None and t.device != q.device:
+            raise ValueError("every tensor must be on q's device")
     sh = make_shape(b, h, g, d, max_chunks * 64, top_k, _dt(q), scale=scale or 0.0)
     if out is None:
         out = torch.empty_like(q)

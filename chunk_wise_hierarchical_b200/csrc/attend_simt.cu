@@ -7,9 +7,12 @@
 // chunk, and d/32 output columns.  The group's G query heads share every key
 // and value load.  For each chunk the warp computes, per head, the running
 // max m, the sum l of exp(s - m) and the unnormalised PV row; the fusion then
-// weights chunk c by exp(shat_c - M) / Z' and the own chunk by
-// exp(LSE_own - M) / Z', with M the max of all log-masses and Z' their
-// shifted sum.
+// weights chunk c by exp(shat_c - M) / Z' and the local branch by
+// exp(LSE_local - M) / Z', with M the max of all log-masses and Z' their
+// shifted sum.  The local branch is the own causal chunk or, with a sliding
+// window of n_local chunks, the own chunk and the n_local - 1 chunks before
+// it, merged chunk by chunk with the split-softmax rule.  The row's log Zhat
+// = M + log Z' is written when an lse buffer is given.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -124,28 +127,43 @@ __global__ void __launch_bounds__(kRowWarps * 32) attend_rows_kernel(AttendRowsA
   };
 
   const int own = pos / B;
-  ChunkAcc<T, D, G> r;
+  const int lo_c = max(0, own + 1 - a.n_local);  // first chunk of the local branch
+  const int n_cand = lo_c;                        // remote candidates: c < lo_c
+  ChunkAcc<T, D, G> r, loc;
   bool ok;
-  const T* kp = chunk_ptr(kb, own, ok);
-  const T* vp = chunk_ptr(vb, own, ok);
   float lse_own[G], acc[G][D / 32];
-  if (!ok) {
-    set_error(a.err, kErrBadPage);
-    for (int hh = 0; hh < G; ++hh)
-      for (int x = 0; x < D / 32; ++x) out_row(hh)[lane + 32 * x] = from_f<T>(0.f);
-    return;
+  // local branch, chunk by chunk (the last one causal up to the query)
+  for (int c = lo_c; c <= own; ++c) {
+    const T* kp = chunk_ptr(kb, c, ok);
+    const T* vp = chunk_ptr(vb, c, ok);
+    if (!ok) {
+      set_error(a.err, kErrBadPage);
+      for (int hh = 0; hh < G; ++hh)
+        for (int x = 0; x < D / 32; ++x) out_row(hh)[lane + 32 * x] = from_f<T>(0.f);
+      return;
+    }
+    chunk_attend<T, D, G>(qS[warp], kp, vp, c == own ? pos - own * B + 1 : B, a.scale, c == lo_c ? loc : r);
+    if (c == lo_c) continue;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {  // merge r into loc
+      const float m = fmaxf(loc.m[hh], r.m[hh]);
+      const float fa = expf(loc.m[hh] - m), fb = expf(r.m[hh] - m);
+      loc.l[hh] = loc.l[hh] * fa + r.l[hh] * fb;
+#pragma unroll
+      for (int x = 0; x < D / 32; ++x) loc.o[hh][x] = loc.o[hh][x] * fa + r.o[hh][x] * fb;
+      loc.m[hh] = m;
+    }
   }
-  chunk_attend<T, D, G>(qS[warp], kp, vp, pos - own * B + 1, a.scale, r);
   const int32_t* idx = a.idx + (((size_t)bi * a.g + gi) * n_q + qi) * K;
   float M[G], Zp[G];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    lse_own[hh] = r.m[hh] + logf(r.l[hh]);
+    lse_own[hh] = loc.m[hh] + logf(loc.l[hh]);
     M[hh] = lse_own[hh];
   }
   // fusion max and normaliser over the selected surrogate masses
   for (int s = 0; s < K; ++s) {
-    if (idx[s] < 0 || (!a.paged && idx[s] >= own)) continue;
+    if (idx[s] < 0 || (!a.paged && idx[s] >= n_cand)) continue;
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       const float sh = a.ssel[(((size_t)bi * a.h + gi * G + hh) * n_q + qi) * K + s];
@@ -155,22 +173,24 @@ __global__ void __launch_bounds__(kRowWarps * 32) attend_rows_kernel(AttendRowsA
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) Zp[hh] = expf(lse_own[hh] - M[hh]);
   for (int s = 0; s < K; ++s) {
-    if (idx[s] < 0 || (!a.paged && idx[s] >= own)) continue;
+    if (idx[s] < 0 || (!a.paged && idx[s] >= n_cand)) continue;
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
       Zp[hh] += expf(a.ssel[(((size_t)bi * a.h + gi * G + hh) * n_q + qi) * K + s] - M[hh]);
   }
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    // own chunk: weight exp(LSE_own - M)/Z', intra part o/l  => o * exp(m - M) / Z'
-    const float w = expf(r.m[hh] - M[hh]) / Zp[hh];
+    // local branch: weight exp(LSE_local - M)/Z', intra part o/l  => o * exp(m - M) / Z'
+    const float w = expf(loc.m[hh] - M[hh]) / Zp[hh];
 #pragma unroll
-    for (int x = 0; x < D / 32; ++x) acc[hh][x] = r.o[hh][x] * w;
+    for (int x = 0; x < D / 32; ++x) acc[hh][x] = loc.o[hh][x] * w;
+    if (a.lse && lane == 0 && !a.paged)
+      a.lse[((size_t)bi * a.h + gi * G + hh) * a.n + qi] = M[hh] + logf(Zp[hh]);
   }
   for (int s = 0; s < K; ++s) {
     const int c = idx[s];
     if (c < 0) continue;
-    if (!a.paged && c >= own) { set_error(a.err, kErrBadPage); continue; }
+    if (!a.paged && c >= n_cand) { set_error(a.err, kErrBadPage); continue; }
     const T* kc = chunk_ptr(kb, c, ok);
     const T* vc = chunk_ptr(vb, c, ok);
     if (!ok) { set_error(a.err, kErrBadPage); continue; }
@@ -210,6 +230,7 @@ static cudaError_t rows_by_group(const AttendRowsArgs& a, cudaStream_t st) {
 }
 
 cudaError_t run_attend_rows(const AttendRowsArgs& a, cudaStream_t st) {
+  if (a.n_local < 1) return cudaErrorInvalidValue;
   if (a.bf16) return a.d == 64 ? rows_by_group<__nv_bfloat16, 64>(a, st) : rows_by_group<__nv_bfloat16, 128>(a, st);
   return a.d == 64 ? rows_by_group<float, 64>(a, st) : rows_by_group<float, 128>(a, st);
 }

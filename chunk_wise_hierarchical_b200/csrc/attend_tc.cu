@@ -696,6 +696,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       pk.y = tc::pack_bf16x2(v.z, v.w);
       *reinterpret_cast<uint2*>(a.out + (((size_t)bi * a.h + head0 + hh) * N + q0 + qo) * D + j4 * 4) = pk;
     }
+    // log Zhat = M + log Z', with (M, 1/Z') left in s_rowm / s_rowz by the own items
+    if (a.lse)
+      for (int r = tid; r < nq * G; r += kThreads)
+        a.lse[((size_t)bi * a.h + head0 + r % G) * N + q0 + r / G] = s_rowm[r] - logf(s_rowz[r]);
   }
   tc::fence_after_sync();
   if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);

@@ -78,4 +78,13 @@ __device__ __forceinline__ void set_error(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
 
+// Remote candidate chunks of the query at position i: the complete chunks before its
+// local branch, c < floor(i / B) + 1 - n_local (n_local = 1: the own chunk only; a
+// sliding window of W keys spans n_local = W / B chunks), capped at the C complete
+// chunks.
+__host__ __device__ __forceinline__ int n_candidates(int i, int n_local, int n_chunks) {
+  const int c = i / kChunk + 1 - n_local;
+  return c < 0 ? 0 : (c < n_chunks ? c : n_chunks);
+}
+
 }  // namespace hils

@@ -14,6 +14,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 256;  // error word + reserved
+constexpr int kMaxWindow = 64 * 128;  // local branch of at most 128 chunks
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -32,9 +33,14 @@ hils_status check_shape(const hils_shape* s, bool need_seq) {
   if (s->head_dim != 64 && s->head_dim != 128) return HILS_ERR_UNSUPPORTED;
   if (s->chunk != hils::kChunk) return HILS_ERR_UNSUPPORTED;
   if (s->top_k > hils::kMaxTopK) return HILS_ERR_UNSUPPORTED;
+  if (s->window < 0 || s->window % s->chunk != 0) return HILS_ERR_INVALID_ARG;
+  if (s->window > kMaxWindow) return HILS_ERR_UNSUPPORTED;
   (void)need_seq;
   return HILS_OK;
 }
+
+// Chunks in the local branch: the own chunk (window 0 or B) or window / B.
+int n_local(const hils_shape* s) { return s->window <= s->chunk ? 1 : s->window / s->chunk; }
 
 float eff_scale(const hils_shape* s) {
   return s->scale == 0.f ? 1.0f / std::sqrt((float)s->head_dim) : s->scale;
@@ -82,26 +88,26 @@ hils_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HIL
 // Prefill attention + fusion for a selection: the tcgen05 kernel for bf16
 // inputs when its shared-memory plan fits the shape, else the row kernel.
 cudaError_t run_prefill_attention(const hils_shape* s, const void* q, const void* k, const void* v,
-                                  const int32_t* idx, const float* ssel, void* out, unsigned* err,
-                                  cudaStream_t cs) {
+                                  const int32_t* idx, const float* ssel, void* out, float* lse,
+                                  unsigned* err, cudaStream_t cs) {
   const bool bf16 = s->dtype == HILS_BF16;
   const int G = s->heads_q / s->heads_kv;
-  if (bf16 && hils::attend_tc_supported(s->head_dim, G, s->top_k, s->seq_len)) {
+  if (bf16 && n_local(s) == 1 && hils::attend_tc_supported(s->head_dim, G, s->top_k, s->seq_len)) {
     hils::TcAttendArgs ta{};
     ta.q = static_cast<const __nv_bfloat16*>(q);
     ta.k = static_cast<const __nv_bfloat16*>(k);
     ta.v = static_cast<const __nv_bfloat16*>(v);
-    ta.idx = idx; ta.ssel = ssel; ta.out = static_cast<__nv_bfloat16*>(out); ta.err = err;
+    ta.idx = idx; ta.ssel = ssel; ta.out = static_cast<__nv_bfloat16*>(out); ta.lse = lse; ta.err = err;
     ta.b = s->batch; ta.h = s->heads_q; ta.g = s->heads_kv; ta.n = s->seq_len; ta.top_k = s->top_k;
     ta.scale = eff_scale(s);
     return hils::run_attend_tc(ta, s->head_dim, cs);
   }
   hils::AttendRowsArgs ar{};
-  ar.q = q; ar.k = k; ar.v = v; ar.idx = idx; ar.ssel = ssel; ar.out = out;
+  ar.q = q; ar.k = k; ar.v = v; ar.idx = idx; ar.ssel = ssel; ar.out = out; ar.lse = lse;
   ar.block_table = nullptr; ar.seq_lens = nullptr; ar.err = err;
   ar.b = s->batch; ar.h = s->heads_q; ar.g = s->heads_kv; ar.n = s->seq_len; ar.d = s->head_dim;
   ar.top_k = s->top_k; ar.max_chunks = 0; ar.n_pages = 0; ar.scale = eff_scale(s); ar.bf16 = bf16;
-  ar.paged = false;
+  ar.paged = false; ar.n_local = n_local(s);
   return hils::run_attend_rows(ar, cs);
 }
 
@@ -122,7 +128,7 @@ const char* hils_status_string(int status) {
   return "unknown status";
 }
 
-int32_t hils_abi_version(void) { return 1; }
+int32_t hils_abi_version(void) { return 2; }
 
 hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) {
   if (!bytes) return HILS_ERR_INVALID_ARG;
@@ -200,11 +206,12 @@ hils_status hils_select(const hils_shape* s, const void* q, const float* kbar, c
   a.err = static_cast<unsigned*>(ws);
   a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
   a.n_chunks = C; a.top_k = s->top_k; a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
+  a.n_local = n_local(s);
   return cuda_status(run_select(a, (cudaStream_t)stream));
 }
 
 hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const void* v,
-                        const void* landmark_q, void* out, int32_t* topk_idx_out, void* ws,
+                        const void* landmark_q, void* out, float* lse_out, int32_t* topk_idx_out, void* ws,
                         size_t ws_bytes, void* stream) {
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
@@ -236,23 +243,24 @@ hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const
     hils::SelectArgs se{};
     se.q = q; se.kbar = kbar; se.hbias = hbias; se.idx = idx; se.score = ssel;
     se.b = s->batch; se.h = s->heads_q; se.g = s->heads_kv; se.n = s->seq_len; se.d = s->head_dim;
-    se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16;
+    se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16; se.n_local = n_local(s);
     se.err = reinterpret_cast<unsigned*>(w);
     if (run_select(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
   }
-  return cuda_status(run_prefill_attention(s, q, k, v, idx, ssel, out, reinterpret_cast<unsigned*>(w), cs));
+  return cuda_status(
+      run_prefill_attention(s, q, k, v, idx, ssel, out, lse_out, reinterpret_cast<unsigned*>(w), cs));
 }
 
 hils_status hils_attend_selected(const hils_shape* s, const void* q, const void* k, const void* v,
-                                 const int32_t* topk_idx, const float* topk_score, void* out, void* ws,
-                                 size_t ws_bytes, void* stream) {
+                                 const int32_t* topk_idx, const float* topk_score, void* out, float* lse_out,
+                                 void* ws, size_t ws_bytes, void* stream) {
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if ((size_t)s->batch * s->seq_len == 0) return HILS_OK;
   if (!q || !k || !v || !out || (s->top_k > 0 && (!topk_idx || !topk_score))) return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HILS_ERR_INVALID_ARG;
   if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
-  return cuda_status(run_prefill_attention(s, q, k, v, topk_idx, topk_score, out,
+  return cuda_status(run_prefill_attention(s, q, k, v, topk_idx, topk_score, out, lse_out,
                                            reinterpret_cast<unsigned*>(ws), (cudaStream_t)stream));
 }
 
@@ -274,7 +282,7 @@ hils_status hils_decode_ex(const hils_shape* s, const void* q, const void* k_pag
   if (summary_dtype != HILS_F32 && summary_dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
   if (summary_dtype == HILS_BF16 && s->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
   if (s->batch == 0) return HILS_OK;
-  if (!hils::decode_supported(s->heads_q, s->head_dim)) return HILS_ERR_UNSUPPORTED;
+  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) != 1) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
@@ -398,7 +406,7 @@ hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if (s->batch == 0) return HILS_OK;
-  if (!hils::decode_supported(s->heads_q, s->head_dim)) return HILS_ERR_UNSUPPORTED;
+  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) != 1) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)

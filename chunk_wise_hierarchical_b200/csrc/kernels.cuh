@@ -31,6 +31,7 @@ struct SelectArgs {
   float* score;           // [b,h,N,K] or nullptr
   unsigned* err;          // sticky error word or nullptr
   int b, h, g, n, d, n_chunks, top_k;
+  int n_local;            // chunks in the local branch (1: own chunk; W / B for a window)
   float scale;
   bool bf16;
 };
@@ -76,10 +77,12 @@ struct AttendRowsArgs {
   const int32_t* idx;          // prefill [b,g,N,K]; decode [b,g,K]
   const float* ssel;           // prefill [b,h,N,K]; decode [b,h,K]
   void* out;                   // like q
+  float* lse;                  // prefill [b,h,N] log Zhat, or nullptr
   const int32_t* block_table;  // decode only
   const int32_t* seq_lens;     // decode only
   unsigned* err;
   int b, h, g, n, d, top_k, max_chunks, n_pages;
+  int n_local;                 // chunks in the local branch (1: own chunk)
   float scale;
   bool bf16;
   bool paged;                  // decode mode
@@ -96,6 +99,7 @@ struct alignas(64) TcAttendArgs {
   const int32_t* idx;          // [b,g,N,K]
   const float* ssel;           // [b,h,N,K]
   __nv_bfloat16* out;          // [b,h,N,d]
+  float* lse;                  // [b,h,N] log Zhat, or nullptr
   unsigned* err;
   int b, h, g, n, top_k;
   float scale;

@@ -36,7 +36,7 @@ __global__ void select_simt_kernel(SelectArgs a, int qt) {
   const int bi = blockIdx.x / (n_qtiles * a.g);
   const int i = qtile * qt + t;
   const bool active = i < a.n;
-  const int n_cand = active ? min(i / kChunk, a.n_chunks) : 0;
+  const int n_cand = active ? n_candidates(i, a.n_local, a.n_chunks) : 0;
 
   // stage q rows of the G heads (fp32)
   for (int hh = 0; hh < G; ++hh) {
@@ -48,7 +48,7 @@ __global__ void select_simt_kernel(SelectArgs a, int qt) {
     }
   }
   int last_i = min(a.n - 1, qtile * qt + qt - 1);
-  const int tile_cand = min(last_i / kChunk, a.n_chunks);
+  const int tile_cand = n_candidates(last_i, a.n_local, a.n_chunks);
 
   int cnt = 0, minpos = 0;
   unsigned long long minkey = ~0ull;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
   const int bi = blockIdx.x / (n_qtiles * a.g);
   const int i = qtile * QT + qo;
   const bool active = i < a.n;
-  const int n_cand = active ? min(i / kChunk, a.n_chunks) : 0;
+  const int n_cand = active ? n_candidates(i, a.n_local, a.n_chunks) : 0;
   const size_t head = (size_t)bi * a.h + gi * G + hh;
   {
     const T* qrow = static_cast<const T*>(a.q) + (head * a.n + (active ? i : 0)) * D;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
     }
   }
   const int last_i = min(a.n - 1, qtile * QT + QT - 1);
-  const int tile_cand = min(last_i / kChunk, a.n_chunks);
+  const int tile_cand = n_candidates(last_i, a.n_local, a.n_chunks);
   unsigned long long L[KP];
   float Sc[KP];
 #pragma unroll

@@ -53,8 +53,8 @@ __global__ void __launch_bounds__(kSelThreads) select_tc_kernel(SelectArgs a) {
   const int q0 = qt * 128;
   const int i = q0 + t;
   const bool active = i < N;
-  const int n_cand = active ? min(i / kChunk, C) : 0;
-  const int tile_cand = min((min(N, q0 + 128) - 1) / kChunk, C);
+  const int n_cand = active ? n_candidates(i, a.n_local, C) : 0;
+  const int tile_cand = n_candidates(min(N, q0 + 128) - 1, a.n_local, C);
 
   // shared memory: Q tile [128 x D] | kbar hi [kNc x D] | kbar lo [kNc x D], 128B-swizzled
   const uint32_t sQ = tc::smem_u32(sm);

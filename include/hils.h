@@ -19,6 +19,13 @@
  * Chunks   chunk = B keys (only 64 is supported).  C = seq_len / B (rounded
  *          down) complete chunks; a trailing partial chunk is never a
  *          candidate, it only serves as the own chunk of its queries.
+ * Local    shape.window selects the local branch whose exact mass joins the
+ *          fusion (notes section 5.3).  0 or B: the query's own causal
+ *          partial chunk, keys [floor(i/B)*B, i]; a multiple W of B: a
+ *          chunk-aligned sliding window (notes section 5.2), the own chunk
+ *          and the W/B - 1 complete chunks before it.  The remote candidates
+ *          of query i are the complete chunks before its local branch,
+ *          c < floor(i/B) + 1 - W/B.
  * Dtype    shape.dtype gives the element type of q, k, v, landmark
  *          queries and out: HILS_BF16 or HILS_F32.  Summaries (kbar,
  *          hbias) and scores are always fp32; indices int32.
@@ -85,12 +92,14 @@ typedef struct {
   int32_t top_k;     /* K, remote chunks kept per query */
   float scale;       /* logit scale; 0 => 1/sqrt(d) */
   int32_t dtype;     /* hils_dtype */
+  int32_t window;    /* local branch: 0 or chunk = own chunk; W = k*chunk =
+                        sliding window of k chunks (see "Local" above) */
 } hils_shape;
 
 /* Static English text for a status code; never NULL. */
 HILS_API const char* hils_status_string(int status);
 
-/* ABI version, currently 1. */
+/* ABI version, currently 2 (1 had no window field and no lse_out). */
 HILS_API int32_t hils_abi_version(void);
 
 /* Bytes of device workspace `op` needs for `shape`, written to *bytes.
@@ -134,9 +143,10 @@ HILS_API hils_status hils_summarize_paged(const hils_shape* shape, const void* k
  * hils_select -- chunk scores and Top-K (notes section 5.2:
  *  shat_{i,c} = q_i.kbar_c * scale + H_c, I_i = the K best candidates;
  *  section 5.4: under GQA the selection key is the max over the group's
- *  query heads).  Candidates of query i are the complete chunks
- *  c < floor(i / B); K_eff = min(K, floor(i / B)).  Ties go to the lower
- *  chunk index.
+ *  query heads).  Candidates of query i are the complete chunks before
+ *  its local branch, c < n_i = floor(i/B) + 1 - W/B (n_i = floor(i/B) for
+ *  the own-chunk branch); K_eff = min(K, max(n_i, 0)).  Ties go to the
+ *  lower chunk index.
  *   q           [batch, heads_q, seq_len, head_dim] (dtype)
  *   kbar, hbias as written by hils_summarize
  *   topk_idx    [batch, heads_kv, seq_len, top_k] int32, written in
@@ -164,12 +174,16 @@ HILS_API hils_status hils_select(const hils_shape* shape, const void* q, const f
  *   q, k, v      prefill layout (dtype)
  *   landmark_q   [batch, heads_q, C, head_dim] (dtype)
  *   out          [batch, heads_q, seq_len, head_dim] (dtype), written
+ *   lse_out      [batch, heads_q, seq_len] fp32 or NULL: log Zhat_i, the
+ *                log-sum-exp of the row's fusion logits (the selected
+ *                chunks' shat and the local branch's exact log-mass), the
+ *                row statistic a backward pass needs
  *   topk_idx_out [batch, heads_kv, seq_len, top_k] int32 or NULL
  *   ws           workspace of hils_workspace_size(HILS_OP_ATTEND) bytes
  */
 HILS_API hils_status hils_attend(const hils_shape* shape, const void* q, const void* k, const void* v,
-                        const void* landmark_q, void* out, int32_t* topk_idx_out, void* ws,
-                        size_t ws_bytes, void* stream);
+                        const void* landmark_q, void* out, float* lse_out, int32_t* topk_idx_out,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /*
  * hils_attend_selected -- the attention half of hils_attend for a selection
@@ -179,24 +193,29 @@ HILS_API hils_status hils_attend(const hils_shape* shape, const void* q, const v
  * inter-chunk softmax of notes section 5.3 (own chunk at its exact mass).
  *   q, k, v      prefill layout (dtype)
  *   topk_idx     [batch, heads_kv, seq_len, top_k] int32; -1 = unused slot;
- *                an entry outside [0, floor(i / B)) is skipped and flagged in
- *                the error word
+ *                an entry that is not a remote candidate of row i (outside
+ *                [0, floor(i/B) + 1 - W/B)) is skipped and flagged in the
+ *                error word
  *   topk_score   [batch, heads_q, seq_len, top_k] fp32: shat of each listed
  *                chunk for each query head
  *   out          [batch, heads_q, seq_len, head_dim] (dtype), written
+ *   lse_out      [batch, heads_q, seq_len] fp32 or NULL: log Zhat_i as in
+ *                hils_attend
  *   ws           workspace of hils_workspace_size(HILS_OP_ATTEND_SELECTED)
  */
 HILS_API hils_status hils_attend_selected(const hils_shape* shape, const void* q, const void* k,
                                           const void* v, const int32_t* topk_idx,
-                                          const float* topk_score, void* out, void* ws,
-                                          size_t ws_bytes, void* stream);
+                                          const float* topk_score, void* out, float* lse_out,
+                                          void* ws, size_t ws_bytes, void* stream);
 
 /*
  * hils_decode -- one decode step per sequence over a paged chunk cache.
  * The new query of sequence b sits at position seq_lens[b]-1 and its key and
  * value are already in the cache.  Own chunk = floor((seq_lens[b]-1)/B);
- * candidates are the chunks before it, scored with the cached summaries;
- * then the same intra-chunk attention and fusion as hils_attend.
+ * the local branch is the own chunk (shape.window 0 or B) or the last
+ * window/B chunks up to the new token; candidates are the complete chunks
+ * before the local branch, scored with the cached summaries; then the same
+ * intra-chunk attention and fusion as hils_attend.
  *   q            [batch, heads_q, head_dim] (dtype)
  *   k_pages,
  *   v_pages      [n_pages, heads_kv, B, head_dim] (dtype)
@@ -242,7 +261,12 @@ HILS_API hils_status hils_decode(const hils_shape* shape, const void* q, const v
  * different host threads) race on it and corrupt each other's results; order
  * them on one stream or with events.  Its ticket counters must start at zero:
  * they are zero when the library's device code is loaded, and each call that
- * completes leaves them at zero again.
+ * completes leaves them at zero again.  A call that returns HILS_ERR_CUDA
+ * after its first kernel was enqueued (the second launch failed) can leave
+ * tickets non-zero; later calls on that device then return wrong results
+ * until the library's device code is loaded again (a new process).
+ * kbar_pages must be the fp32 summary cache (this entry point has no
+ * summary_dtype argument).
  */
 #define HILS_DECODE_STATIC_SCRATCH_BYTES (4u << 20)
 HILS_API hils_status hils_decode_static(const hils_shape* shape, const void* q, const void* k_pages,

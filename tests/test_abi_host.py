@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     lib = hils.lib()
-    assert lib.hils_abi_version() == 1
+    assert lib.hils_abi_version() == 2
     for code in range(7):
         assert lib.hils_status_string(code)
     assert lib.hils_status_string(99) == b"unknown status"
@@ -39,7 +39,8 @@ def _shape(**kw):
     base.update(kw)
     return _abi.make_shape(base["batch"], base["heads_q"], base["heads_kv"], base["head_dim"],
                            base["seq_len"], base["top_k"], base["dtype"],
-                           chunk=base.get("chunk", 64), scale=base.get("scale", 0.0))
+                           chunk=base.get("chunk", 64), scale=base.get("scale", 0.0),
+                           window=base.get("window", 0))
 
 
 def test_workspace_sizes():
@@ -56,6 +57,8 @@ def test_workspace_sizes():
     (dict(head_dim=96), 2), (dict(chunk=32), 2), (dict(top_k=65), 2), (dict(heads_q=6, heads_kv=2), 2),
     (dict(heads_q=7, heads_kv=2), 1), (dict(batch=-1), 1), (dict(dtype=5), 1), (dict(top_k=-1), 1),
     (dict(scale=float("nan")), 1), (dict(heads_q=32, heads_kv=2), 2),
+    (dict(window=-64), 1), (dict(window=100), 1), (dict(window=64 * 129), 2), (dict(window=512), 0),
+    (dict(window=64), 0),
 ])
 def test_shape_validation(kw, code):
     s = _shape(**kw)
@@ -69,11 +72,13 @@ def test_entry_points_reject_before_launch():
     P = ctypes.c_void_p
     fake = P(1 << 20)  # never dereferenced: every call below fails validation first
     assert lib.hils_workspace_size(None, 1, ctypes.byref(ctypes.c_size_t())) == 1
-    assert lib.hils_attend(ctypes.byref(s), None, fake, fake, fake, fake, None, fake, 1 << 30, None) == 1
-    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, None, 0, None) == 3
-    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, fake, 16, None) == 3
-    assert lib.hils_attend(ctypes.byref(s), P((1 << 20) + 4), fake, fake, fake, fake, None, fake,
+    assert lib.hils_attend(ctypes.byref(s), None, fake, fake, fake, fake, None, None, fake, 1 << 30, None) == 1
+    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, None, None, 0, None) == 3
+    assert lib.hils_attend(ctypes.byref(s), fake, fake, fake, fake, fake, None, None, fake, 16, None) == 3
+    assert lib.hils_attend(ctypes.byref(s), P((1 << 20) + 4), fake, fake, fake, fake, None, None, fake,
                            1 << 30, None) == 1  # misaligned
+    assert lib.hils_attend_selected(ctypes.byref(s), fake, fake, fake, None, fake, fake, None, fake,
+                                    1 << 30, None) == 1  # top_k > 0 without indices
     assert lib.hils_select(ctypes.byref(s), fake, None, fake, fake, None, None, 0, None) == 1
     assert lib.hils_select(ctypes.byref(s), fake, fake, fake, fake, None, None, 0, None) == 3  # no error word
     assert lib.hils_summarize(ctypes.byref(s), fake, None, fake, fake, None) == 1
@@ -89,11 +94,11 @@ def test_empty_problems_are_no_ops():
     lib = hils.lib()
     P = ctypes.c_void_p
     s0 = _shape(batch=0)
-    assert lib.hils_attend(ctypes.byref(s0), None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.hils_attend(ctypes.byref(s0), None, None, None, None, None, None, None, None, 0, None) == 0
     assert lib.hils_decode(ctypes.byref(s0), None, None, None, None, None, None, 0, None, 0, None, None,
                            None, 0, None) == 0
     s1 = _shape(seq_len=0)
-    assert lib.hils_attend(ctypes.byref(s1), None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.hils_attend(ctypes.byref(s1), None, None, None, None, None, None, None, None, 0, None) == 0
     assert lib.hils_summarize(ctypes.byref(s1), None, None, None, None, None) == 0
     s2 = _shape(top_k=0)
     assert lib.hils_select(ctypes.byref(s2), None, None, None, None, None, None, 0, None) == 0
@@ -121,3 +126,26 @@ def test_summary_dtype_validation():
     assert lib.hils_summarize_paged_ex(ctypes.byref(s_f32), fake, fake, fake, 4, 4, fake, 1, fake, None) == 2
     assert lib.hils_decode_ex(ctypes.byref(s_f32), fake, fake, fake, fake, 1, fake, fake, 1, fake, 4, fake,
                               None, fake, 1 << 30, None) == 2
+
+
+def test_decode_with_a_window_is_not_yet_supported_by_the_decode_kernels():
+    lib = hils.lib()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the call fails validation first
+    s = _shape(window=512, seq_len=4096)
+    assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 8, fake, 4, fake, None,
+                           fake, 1 << 30, None) == 2
+
+
+def test_decode_static_binding_rejects_a_bf16_summary_cache():
+    """hils_decode_static reads fp32 summaries only: the binding refuses a bf16
+    cache before any pointer reaches the library."""
+    import torch
+    q = torch.zeros(2, 4, 64, dtype=torch.bfloat16)
+    kp = torch.zeros(3, 2, 64, 64, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 1, dtype=torch.int32)
+    sl = torch.ones(2, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        hils.decode_static(q, kp, kp, torch.zeros(3, 4, 64, dtype=torch.bfloat16), torch.zeros(3, 4), bt, sl, 2)
+    with pytest.raises(TypeError):
+        hils.decode_static(q, kp, kp, torch.zeros(3, 4, 64), torch.zeros(3, 4), bt, sl, 2,
+                           topk_idx=torch.zeros(2, 2, 2, dtype=torch.int64))

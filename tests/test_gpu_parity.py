@@ -22,27 +22,36 @@ def _np(t):
     return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
 
 
-def _prefill_case(rows=None, heads=None, **kw):
+LSE_TOL = {True: 2e-3, False: 1e-4}  # log Zhat, bf16 / fp32 inputs (fp32 arithmetic either way)
+
+
+def _prefill_case(rows=None, heads=None, window=0, **kw):
     inp = prefill_inputs(device="cpu", **kw)
     q, k, v, lm = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.landmark))
     K = inp.top_k
-    out, idx = hils.attend(q, k, v, lm, K, return_idx=True)
+    out, idx, lse = hils.attend(q, k, v, lm, K, return_idx=True, return_lse=True, window=window)
     torch.cuda.synchronize()
     n = q.shape[2]
     rows = np.arange(n) if rows is None else np.asarray(rows)
-    ref = O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, K, rows=rows, heads=heads)
+    win = window or None
+    ref = O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, K, rows=rows, heads=heads, window=win)
     gidx = idx.cpu().numpy()[:, :, rows]
     ties = check_indices(gidx, ref["key"], K)
     if not np.array_equal(gidx, ref["idx"]):
         ref = O.forward(inp.q, inp.k, inp.v, inp.landmark, 64, K, rows=rows, heads=heads,
-                        forced_idx=gidx)
+                        forced_idx=gidx, window=win)
     got = _np(out)[:, :, rows]
     want = ref["out"]
+    got_lse = lse.cpu().numpy()[:, :, rows]
+    want_lse = ref["lse"]
     if heads is not None:
         sel = tuple(np.array(heads).T)
         got, want = got[sel], want[sel]
+        got_lse, want_lse = got_lse[sel], want_lse[sel]
     bf16 = inp.q.dtype == torch.bfloat16
     err = check_close(got, want, bf16)
+    lse_err = np.abs(got_lse - want_lse).max()
+    assert lse_err <= LSE_TOL[bf16], f"log Zhat max abs err {lse_err:.3g}"
     return inp, idx, ties, err
 
 
@@ -146,12 +155,24 @@ def _rows_sample(n, rng, count=40):
     return np.unique(np.concatenate([edge, rng.integers(0, n, count)]))
 
 
+def _needle_recall(inp, idx, group):
+    """Diagnostic (not parity): the fraction of planted needles whose target query
+    selected the needle's chunk.  Printed, not asserted: with N(0,1) landmark queries
+    the needle barely moves its chunk's summary, so recall is near what the needle's
+    own logit buys, and the oracle's recall is the same on the same data."""
+    gi = idx.cpu().numpy()
+    hits = sum(int(c in gi[b, h // group, i]) for b, h, c, j, i in inp.needles)
+    print(f"needle recall: {hits} of {len(inp.needles)}")
+    return hits
+
+
 def test_prefill_345m_full_size_sampled():
     cfg = CONFIGS["prefill_345m"]
     rng = np.random.default_rng(1)
     rows = _rows_sample(cfg["seq_len"], rng)
     heads = [(0, 0), (1, 7), (3, 15)]
-    _prefill_case(rows=rows, heads=heads, seed=0, **cfg)
+    inp, idx, _, _ = _prefill_case(rows=rows, heads=heads, seed=0, **cfg)
+    _needle_recall(inp, idx, 1)
 
 
 def test_prefill_7b_gqa_full_size_sampled():
@@ -159,7 +180,19 @@ def test_prefill_7b_gqa_full_size_sampled():
     rng = np.random.default_rng(2)
     rows = _rows_sample(cfg["seq_len"], rng, count=24)
     heads = [(0, 0), (0, 13), (0, 31)]
-    _prefill_case(rows=rows, heads=heads, seed=0, **cfg)
+    inp, idx, _, _ = _prefill_case(rows=rows, heads=heads, seed=0, **cfg)
+    _needle_recall(inp, idx, 4)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(batch=1, heads_q=2, heads_kv=2, seq_len=64 * 20 + 9, head_dim=64, top_k=4, dtype="bf16", window=256),
+    dict(batch=1, heads_q=4, heads_kv=1, seq_len=64 * 14, head_dim=128, top_k=3, dtype="f32", window=192),
+    dict(batch=2, heads_q=8, heads_kv=2, seq_len=64 * 12 + 40, head_dim=64, top_k=8, dtype="bf16", window=512),
+    dict(batch=1, heads_q=2, heads_kv=2, seq_len=300, head_dim=64, top_k=2, dtype="f32", window=64),
+])
+def test_prefill_sliding_window_local_branch(kw):
+    """The chunk-aligned sliding-window local branch (notes sections 5.2-5.3)."""
+    _prefill_case(seed=13, **kw)
 
 
 # --------------------------------------------------------------------------- decode
@@ -259,6 +292,15 @@ def test_decode_32k_full_size_sampled():
     di = decode_inputs(device="cuda", seed=0, **cfg)
     out, idx = _gpu_decode(di, cfg["top_k"])
     _check_decode(di, out, idx, cfg["top_k"], [(0, 0), (7, 5), (3, 15)])
+
+
+def test_decode_128k_full_size_sampled():
+    cfg = CONFIGS["decode_128k"]
+    di = decode_inputs(device="cuda", seed=0, **cfg)
+    out, idx = _gpu_decode(di, cfg["top_k"])
+    _check_decode(di, out, idx, cfg["top_k"], [(1, 2), (6, 11)])
+    del di
+    torch.cuda.empty_cache()
 
 
 def test_decode_512k_full_size_sampled():
@@ -363,3 +405,61 @@ def test_decode_with_bf16_summary_cache(kw):
                 check_indices(gi[None], ref["key"][0][0][None], K, gap=2 * bound + 1e-3)
             want = _forced_decode(q, kps, vps, lps, bt, sl, gi) if sl[0] > 64 else ref["out"][0]
             check_close(_np(out[b, gsel * grp:(gsel + 1) * grp]), want, True)
+
+
+def _outside_band(gpu_idx, key, top_k, gap):
+    """True when the GPU selection breaks the Top-K gap rule at `gap`."""
+    try:
+        check_indices(gpu_idx, key, top_k, gap=gap)
+        return False
+    except AssertionError:
+        return True
+
+
+@pytest.mark.parametrize("name,pairs", [
+    ("decode_32k", [(0, 0), (1, 3), (2, 6), (3, 9), (4, 12), (5, 15), (6, 1), (7, 4)]),
+    ("decode_128k", [(0, 2), (3, 7), (5, 11), (7, 14)]),
+    ("decode_512k", [(2, 3), (6, 10)]),
+])
+def test_bf16_summary_cache_against_the_gap_rule_at_full_size(name, pairs):
+    """The compact bf16 summary cache judged by the 1e-3 Top-K gap rule.
+
+    Reported: how many sampled (sequence, KV head) selections differ from the
+    oracle's outside the 1e-3 band (the bf16 rounding of kbar can move a score by
+    up to scale * 2^-8 * sum |q||kbar|, well above 1e-3).  Asserted: the selection
+    holds outside the band that rounding allows (2 * bound + 1e-3), and the output
+    matches the oracle fused over the GPU's selection."""
+    cfg = CONFIGS[name]
+    K = cfg["top_k"]
+    di = decode_inputs(device="cuda", seed=0, **cfg)
+    P, g, B, d = di.k_pages.shape
+    h = di.landmark_pages.shape[1]
+    ids = torch.arange(P, dtype=torch.int32, device="cuda")
+    kbar16 = torch.empty((P, h, d), dtype=torch.bfloat16, device="cuda")
+    kbar32 = torch.empty((P, h, d), dtype=torch.float32, device="cuda")
+    hb = torch.empty((P, h), dtype=torch.float32, device="cuda")
+    hils.summarize_paged(di.k_pages, di.landmark_pages, ids, kbar16, hb)
+    hils.summarize_paged(di.k_pages, di.landmark_pages, ids, kbar32, torch.empty_like(hb))
+    out, idx = hils.decode(di.q, di.k_pages, di.v_pages, kbar16, hb, di.block_table, di.seq_lens, K,
+                           return_idx=True)
+    torch.cuda.synchronize()
+    scale = 1.0 / np.sqrt(d)
+    grp = h // g
+    outside = 0
+    for b, gsel in pairs:
+        q, kps, vps, lps, bt, sl = _slice_for_oracle(di, b, gsel)
+        ref = O.decode(q, kps, vps, lps, bt, sl, K)
+        gi = idx[b, gsel].cpu().numpy()
+        key = ref["key"][0][0][None]
+        outside += _outside_band(gi[None], key, K, 1e-3)
+        pages = di.block_table[b].long()[: (sl[0] - 1) // 64]
+        qa = di.q[b, gsel * grp:(gsel + 1) * grp].double().abs()
+        ka = kbar32[pages][:, gsel * grp:(gsel + 1) * grp].double().abs()
+        bound = float((qa[None] * ka).sum(-1).max()) * scale * 2.0 ** -8
+        check_indices(gi[None], key, K, gap=2 * bound + 1e-3)
+        want = _forced_decode(q, kps, vps, lps, bt, sl, gi)
+        check_close(_np(out[b, gsel * grp:(gsel + 1) * grp]), want, True)
+    print(f"{name}: bf16 summary cache, {outside} of {len(pairs)} sampled selections differ from the "
+          f"oracle's outside the 1e-3 gap band")
+    del di
+    torch.cuda.empty_cache()
