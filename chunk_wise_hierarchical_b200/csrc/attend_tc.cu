@@ -752,6 +752,7 @@ static int pick_qb(int G, int K, int N, size_t* smem_out) {
 bool attend_tc_supported(int d, int G, int K, int N) {
   size_t smem;
   if (K > 64 || N / kChunk > 32767 || tensor_map_encoder() == nullptr) return false;
+  if (d == 64 && attend_tc3_supported(d, G, K, N)) return true;
   return d == 64 ? pick_qb<64>(G, K, N, &smem) > 0 : d == 128 ? pick_qb<128>(G, K, N, &smem) > 0 : false;
 }
 
@@ -785,6 +786,12 @@ static cudaError_t tc_by_group(const TcAttendArgs& a, cudaStream_t st) {
 }
 
 cudaError_t run_attend_tc(const TcAttendArgs& a, int d, cudaStream_t st) {
+  if (d == 64 && attend_tc3_supported(d, a.h / a.g, a.top_k, a.n)) {
+    TcAttendArgs b = a;
+    if (!encode_kv_map(&b.tmap_k, b.k, 64, b.n, b.b * b.g) || !encode_kv_map(&b.tmap_v, b.v, 64, b.n, b.b * b.g))
+      return cudaErrorNotSupported;
+    return run_attend_tc3(b, st);
+  }
   return d == 64 ? tc_by_group<64>(a, st) : tc_by_group<128>(a, st);
 }
 

@@ -108,5 +108,8 @@ struct alignas(64) TcAttendArgs {
 };
 bool attend_tc_supported(int d, int G, int K, int N);
 cudaError_t run_attend_tc(const TcAttendArgs& a, int d, cudaStream_t st);
+// Head dim 64: Q rows in tensor memory, conflict-free accumulation order (tensor maps set).
+bool attend_tc3_supported(int d, int G, int K, int N);
+cudaError_t run_attend_tc3(const TcAttendArgs& a, cudaStream_t st);
 
 }  // namespace hils
