@@ -10,11 +10,13 @@ from ._abi import (  # noqa: F401
     Decode,
     attend,
     attend_selected,
+    backward,
     new_workspace,
     OP_SELECT,
     OP_ATTEND,
     OP_DECODE,
     OP_ATTEND_SELECTED,
+    OP_BACKWARD,
     decode,
     decode_static,
     select,

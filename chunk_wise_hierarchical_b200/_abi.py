@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhils.so")
 
 HILS_F32, HILS_BF16 = 0, 1
-OP_SELECT, OP_ATTEND, OP_DECODE, OP_ATTEND_SELECTED = 0, 1, 2, 3
+OP_SELECT, OP_ATTEND, OP_DECODE, OP_ATTEND_SELECTED, OP_BACKWARD = 0, 1, 2, 3, 4
 STATUS = {
     0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED", 3: "HILS_ERR_WORKSPACE",
     4: "HILS_ERR_CUDA", 5: "HILS_ERR_DEVICE_CHECK", 6: "HILS_ERR_DEVICE_TIMEOUT",
@@ -70,6 +70,7 @@ def lib():
         "hils_decode_ex": (i32, [S, _P, _P, _P, _P, i32, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
         "hils_decode_static": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, _P]),
         "hils_device_status": (i32, [_P, _P]),
+        "hils_backward": (i32, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -79,7 +80,7 @@ def lib():
     return L
 
 
-EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_decode",
+EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_backward", "hils_decode",
             "hils_decode_ex", "hils_decode_static", "hils_device_status", "hils_summarize_paged_ex", "hils_select", "hils_status_string", "hils_summarize",
             "hils_summarize_paged", "hils_workspace_size"]
 
@@ -325,3 +326,37 @@ def decode_static(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq
                                     int(k_pages.shape[0]), _ptr(out), _ptr(topk_idx), _ptr(status_word),
                                     _stream(stream)), "hils_decode_static")
     return out
+
+
+def backward(q, k, v, landmark, out, lse, topk_idx, topk_score, dout, scale=None, window=0, stream=None,
+             ws=None):
+    """hils_backward: fp32 (dq, dk, dv, dlandmark) for the forward that produced out,
+    lse (log Zhat), topk_idx and topk_score on these bf16 inputs."""
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    K = topk_idx.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("hils_backward takes bf16 inputs")
+    for t in (k, v, landmark, out, dout):
+        if t.dtype != torch.bfloat16:
+            raise TypeError("q, k, v, landmark, out and dout must be bf16")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must have q's shape")
+    if lse.dtype != torch.float32 or lse.shape != (b, h, n):
+        raise ValueError("lse must be fp32 [b, h, N]")
+    if topk_idx.dtype != torch.int32 or topk_idx.shape != (b, g, n, K):
+        raise ValueError("topk_idx must be int32 [b, heads_kv, N, K]")
+    if topk_score.dtype != torch.float32 or topk_score.shape != (b, h, n, K):
+        raise ValueError("topk_score must be fp32 [b, heads_q, N, K]")
+    sh = make_shape(b, h, g, d, n, K, HILS_BF16, scale=scale or 0.0, window=window)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((b, h, n, d), **f32)
+    dk = torch.empty((b, g, n, d), **f32)
+    dv = torch.empty((b, g, n, d), **f32)
+    dl = torch.zeros(landmark.shape, **f32)
+    if ws is None:
+        ws = new_workspace(sh, OP_BACKWARD, q.device)
+    _check(lib().hils_backward(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), _ptr(landmark), _ptr(out), _ptr(lse),
+                               _ptr(topk_idx), _ptr(topk_score), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(dl), _ptr(ws), ws.numel(), _stream(stream)), "hils_backward")
+    return dq, dk, dv, dl

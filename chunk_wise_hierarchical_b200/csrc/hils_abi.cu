@@ -62,6 +62,21 @@ AttendLayout attend_layout(const hils_shape* s) {
   return L;
 }
 
+struct BackwardLayout {
+  size_t drow, list_off, list, total;
+};
+BackwardLayout backward_layout(const hils_shape* s) {
+  const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, n = s->seq_len, K = s->top_k;
+  const size_t C = n / s->chunk;
+  BackwardLayout L;
+  size_t off = kHeader;
+  L.drow = off; off = align_up(off + b * h * n * 4);
+  L.list_off = off; off = align_up(off + b * g * (C + 1) * 4);
+  L.list = off; off = align_up(off + b * g * n * K * 4);
+  L.total = off;
+  return L;
+}
+
 struct DecodeLayout {
   size_t part_keys, part_att, scan_ticket, att_ticket, idx, sel_page, ssel, total;
 };
@@ -139,6 +154,7 @@ hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) 
     case HILS_OP_ATTEND: *bytes = attend_layout(s).total; return HILS_OK;
     case HILS_OP_DECODE: *bytes = decode_layout(s).total; return HILS_OK;
     case HILS_OP_ATTEND_SELECTED: *bytes = kHeader; return HILS_OK;
+    case HILS_OP_BACKWARD: *bytes = backward_layout(s).total; return HILS_OK;
   }
   return HILS_ERR_INVALID_ARG;
 }
@@ -262,6 +278,37 @@ hils_status hils_attend_selected(const hils_shape* s, const void* q, const void*
   if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
   return cuda_status(run_prefill_attention(s, q, k, v, topk_idx, topk_score, out, lse_out,
                                            reinterpret_cast<unsigned*>(ws), (cudaStream_t)stream));
+}
+
+hils_status hils_backward(const hils_shape* s, const void* q, const void* k, const void* v,
+                          const void* landmark_q, const void* out, const float* lse, const int32_t* topk_idx,
+                          const float* topk_score, const void* dout, float* dq, float* dk, float* dv,
+                          float* dlandmark, void* ws, size_t ws_bytes, void* stream) {
+  hils_status st = check_shape(s, true);
+  if (st != HILS_OK) return st;
+  if (s->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
+  if ((size_t)s->batch * s->seq_len == 0) return HILS_OK;
+  if ((long long)s->seq_len * s->top_k >= (1ll << 31) || s->seq_len >= (1 << 25)) return HILS_ERR_UNSUPPORTED;
+  const int C = s->seq_len / s->chunk;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return HILS_ERR_INVALID_ARG;
+  if (C > 0 && (!landmark_q || !dlandmark)) return HILS_ERR_INVALID_ARG;
+  if (s->top_k > 0 && (!topk_idx || !topk_score)) return HILS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (C > 0 && !aligned16(landmark_q)))
+    return HILS_ERR_INVALID_ARG;
+  const BackwardLayout L = backward_layout(s);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
+  hils::BwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.landmark = landmark_q; a.out = out; a.dout = dout; a.lse = lse;
+  a.idx = topk_idx; a.ssel = topk_score; a.dq = dq; a.dk = dk; a.dv = dv; a.dlandmark = dlandmark;
+  a.drow = reinterpret_cast<float*>(w + L.drow);
+  a.list_off = reinterpret_cast<int*>(w + L.list_off);
+  a.list = reinterpret_cast<int*>(w + L.list);
+  a.err = reinterpret_cast<unsigned*>(w);
+  a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
+  a.top_k = s->top_k; a.n_local = n_local(s); a.scale = eff_scale(s);
+  return cuda_status(hils::run_backward(a, (cudaStream_t)stream));
 }
 
 hils_status hils_decode(const hils_shape* s, const void* q, const void* k_pages, const void* v_pages,

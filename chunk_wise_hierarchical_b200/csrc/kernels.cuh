@@ -106,6 +106,30 @@ struct alignas(64) TcAttendArgs {
   int qb;                      // queries per CTA (set by the launcher)
   int n_cand_max;              // N / chunk (set by the launcher)
 };
+// Backward pass (bf16 inputs, fp32 gradients) for a forward's selection and row normaliser.
+struct BwdArgs {
+  const void* q;          // [b,h,N,d] bf16
+  const void* k;          // [b,g,N,d]
+  const void* v;
+  const void* landmark;   // [b,h,C,d]
+  const void* out;        // [b,h,N,d] forward output
+  const void* dout;       // [b,h,N,d] upstream gradient
+  const float* lse;       // [b,h,N] log Zhat of the forward
+  const int32_t* idx;     // [b,g,N,K]
+  const float* ssel;      // [b,h,N,K] shat of the selected chunks
+  float* dq;              // [b,h,N,d] (accumulated: cleared by the launcher)
+  float* dk;              // [b,g,N,d]
+  float* dv;
+  float* dlandmark;       // [b,h,C,d]
+  float* drow;            // workspace [b,h,N]: dO . o
+  int* list_off;          // workspace [b,g,C+1]
+  int* list;              // workspace [b,g,N*K]
+  unsigned* err;
+  int b, h, g, n, d, top_k, n_local;
+  float scale;
+};
+cudaError_t run_backward(const BwdArgs& a, cudaStream_t st);
+
 bool attend_tc_supported(int d, int G, int K, int N);
 cudaError_t run_attend_tc(const TcAttendArgs& a, int d, cudaStream_t st);
 // Head dim 64: Q rows in tensor memory, conflict-free accumulation order (tensor maps set).

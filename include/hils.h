@@ -79,7 +79,8 @@ typedef enum {
   HILS_OP_SELECT = 0,
   HILS_OP_ATTEND = 1,
   HILS_OP_DECODE = 2,
-  HILS_OP_ATTEND_SELECTED = 3
+  HILS_OP_ATTEND_SELECTED = 3,
+  HILS_OP_BACKWARD = 4
 } hils_op;
 
 typedef struct {
@@ -207,6 +208,36 @@ HILS_API hils_status hils_attend_selected(const hils_shape* shape, const void* q
                                           const void* v, const int32_t* topk_idx,
                                           const float* topk_score, void* out, float* lse_out,
                                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * hils_backward -- gradients of the prefill forward pass (hils_attend) with
+ * respect to q, k, v and the landmark queries, for an upstream gradient dout
+ * (notes section 5.3: the hierarchical softmax carries the loss into the
+ * chunk scores, so the selector is trained by it; Tide Figure 3 caption: the
+ * gradients reach the compressed key).  The Top-K selection of the forward is
+ * held fixed; every other step is differentiated exactly: the intra-chunk and
+ * local softmaxes, the inter-chunk softmax over shat and the local log-mass,
+ * shat = q.kbar * scale + H, and the landmark softmax that makes kbar and H
+ * (notes section 5.1).  Unselected chunks receive gradient only through the
+ * local branches that contain them.
+ *   q, k, v, landmark_q   the forward's inputs (bf16 only: HILS_ERR_UNSUPPORTED
+ *                         for HILS_F32)
+ *   out                   [batch, heads_q, seq_len, head_dim] bf16, the forward's output
+ *   lse                   [batch, heads_q, seq_len] fp32, the forward's lse_out
+ *   topk_idx, topk_score  the forward's selection and each head's shat of it
+ *                         (hils_select's outputs); may be NULL when top_k == 0
+ *   dout                  [batch, heads_q, seq_len, head_dim] bf16
+ *   dq                    [batch, heads_q, seq_len, head_dim] fp32, written
+ *   dk, dv                [batch, heads_kv, seq_len, head_dim] fp32, written
+ *   dlandmark             [batch, heads_q, C, head_dim] fp32, written
+ *   ws                    workspace of hils_workspace_size(HILS_OP_BACKWARD)
+ * Selection entries outside row i's candidates are skipped and flagged.
+ */
+HILS_API hils_status hils_backward(const hils_shape* shape, const void* q, const void* k, const void* v,
+                          const void* landmark_q, const void* out, const float* lse,
+                          const int32_t* topk_idx, const float* topk_score, const void* dout,
+                          float* dq, float* dk, float* dv, float* dlandmark, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /*
  * hils_decode -- one decode step per sequence over a paged chunk cache.

@@ -149,3 +149,19 @@ def test_decode_static_binding_rejects_a_bf16_summary_cache():
     with pytest.raises(TypeError):
         hils.decode_static(q, kp, kp, torch.zeros(3, 4, 64), torch.zeros(3, 4), bt, sl, 2,
                            topk_idx=torch.zeros(2, 2, 2, dtype=torch.int64))
+
+
+def test_backward_rejects_before_launch():
+    lib = hils.lib()
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: every call below fails validation first
+    s16 = _shape(dtype=1)
+    s32 = _shape(dtype=0)
+    args = [fake] * 13  # q k v landmark out lse idx score dout dq dk dv dl
+    assert lib.hils_backward(ctypes.byref(s32), *args, fake, 1 << 30, None) == 2  # bf16 only
+    no_lse = list(args)
+    no_lse[5] = None
+    assert lib.hils_backward(ctypes.byref(s16), *no_lse, fake, 1 << 30, None) == 1
+    assert lib.hils_backward(ctypes.byref(s16), *args, None, 0, None) == 3
+    n = ctypes.c_size_t(0)
+    assert lib.hils_workspace_size(ctypes.byref(s16), 4, ctypes.byref(n)) == 0 and n.value > 256
