@@ -17,6 +17,7 @@ the data path); rank 0 prints one JSON line with the max time over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -483,6 +484,50 @@ def run_prefill_gqa(dev, steps=5, warmup=3):
             "timing": "CUDA events per stage, median of %d steps, L2 flushed between steps" % steps}
 
 
+def run_training(dev, steps=5, warmup=3):
+    """The training workload (b2 h16 N16384 d128 K16, bf16): one forward (summaries,
+    selection, attention with log Zhat) and one hils_backward per step, with dO ~ N(0,1).
+    Backward algorithmic FLOPs = 2.5 x the forward's: per (query, key) pair the forward
+    does 4d (QK^T, PV) and the backward 10d (QK^T and dO V^T recomputed, dV, dK, dQ)."""
+    import chunk_wise_hierarchical_b200 as hils
+    cfg = CONFIGS["train_16k"]
+    inp = prefill_inputs(seed=0, device=dev, **cfg)
+    q, k, v, lm = inp.q, inp.k, inp.v, inp.landmark
+    b, h, n, d = q.shape
+    g = k.shape[1]
+    K = cfg["top_k"]
+    dout = torch.randn(q.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(1)).to(torch.bfloat16)
+    lse = torch.empty((b, h, n), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    sh = hils.make_shape(b, h, g, d, n, K, 1)
+    ws = hils.new_workspace(sh, hils.OP_BACKWARD, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    for it in range(warmup + steps):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        kbar, hb = hils.summarize(k, lm)
+        idx, sc = hils.select(q, kbar, hb, K, g)
+        hils.attend_selected(q, k, v, idx, sc, out=out, lse=lse)
+        ev[1].record()
+        hils.backward(q, k, v, lm, out, lse, idx, sc, dout, ws=ws)
+        ev[2].record()
+        torch.cuda.synchronize()
+        if it >= warmup:
+            times.append((ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])))
+    assert hils.lib().hils_device_status(ctypes.c_void_p(ws.data_ptr()), None) == 0
+    fwd = statistics.median(t[0] for t in times)
+    bwd = statistics.median(t[1] for t in times)
+    flops = algorithmic_flops(b, h, n, d, K)
+    return {"workload": "train_16k: batch 2, 16 heads, N 16384, d 128, top-k 16, bf16 N(0,1), dO N(0,1)",
+            "forward_ms": round(fwd, 3), "backward_ms": round(bwd, 3),
+            "forward_tflops": round(flops / (fwd * 1e-3) / 1e12, 2),
+            "backward_tflops": round(2.5 * flops / (bwd * 1e-3) / 1e12, 2),
+            "algorithmic_gflop": {"forward": round(flops / 1e9, 1), "backward": round(2.5 * flops / 1e9, 1)},
+            "timing": "CUDA events, median of %d steps, L2 flushed between steps" % steps}
+
+
 # ---------------------------------------------------------------------------- decode (ours)
 def run_decode(name, n_caches, dev, reps=50):
     """Decode step time for the fp32 summary cache and for the compact bf16 one, on the
@@ -560,6 +605,7 @@ def run_ours(args):
         return
     pre = run_prefill(args, ws_world, rank, local)
     gqa = run_prefill_gqa(torch.device("cuda", local)) if not args.no_gqa else None
+    train = run_training(torch.device("cuda", local)) if not args.no_train else None
     cpu = cpu1 = otimes = None
     if rank == 0 and ws_world == 1 and not args.no_cpu:
         cpu = cpu_baseline(args.cpu_seconds)                 # every host core
@@ -610,6 +656,8 @@ def run_ours(args):
     }
     if gqa:
         line["prefill_7b_gqa"] = gqa
+    if train:
+        line["train_16k"] = train
     if dec:
         line["decode"] = {
             k: {"tok_s": round(r["tok_s"], 1), "us_per_step": round(r["ms"] * 1e3, 2),
@@ -668,6 +716,7 @@ def main():
     ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the 7B-shaped GQA prefill line")
+    ap.add_argument("--no-train", action="store_true", help="skip the forward + backward training line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the attention kernel from an ncu capture")

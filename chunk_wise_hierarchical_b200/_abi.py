@@ -257,11 +257,11 @@ class Decode:
     """Reusable decode call for a paged cache of `max_chunks` chunks per sequence."""
 
     def __init__(self, batch, heads_q, heads_kv, head_dim, max_chunks, top_k, dtype, scale=None,
-                 device="cuda"):
+                 device="cuda", window=0):
         self.max_chunks = max_chunks
         self.shape = make_shape(batch, heads_q, heads_kv, head_dim, max_chunks * 64, top_k,
                                 HILS_BF16 if dtype in (torch.bfloat16, "bf16") else HILS_F32,
-                                scale=scale or 0.0)
+                                scale=scale or 0.0, window=window)
         self.ws = new_workspace(self.shape, OP_DECODE, device)
 
     def __call__(self, q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, out=None,
@@ -284,10 +284,10 @@ class Decode:
 
 
 def decode(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, top_k, scale=None,
-           stream=None, return_idx=False):
+           stream=None, return_idx=False, window=0):
     b, h, d = q.shape
     g = k_pages.shape[1]
-    call = Decode(b, h, g, d, block_table.shape[1], top_k, q.dtype, scale=scale, device=q.device)
+    call = Decode(b, h, g, d, block_table.shape[1], top_k, q.dtype, scale=scale, device=q.device, window=window)
     idx = torch.empty((b, g, top_k), dtype=torch.int32, device=q.device) if return_idx else None
     out = call(q, k_pages, v_pages, kbar_pages, hbias_pages, block_table, seq_lens, topk_idx=idx,
                stream=stream)

@@ -33,6 +33,7 @@ constexpr int kMergeN = 256;            // keys one warp sorts at once in the fa
 
 
 constexpr int kMaxListsPerLane = 4;
+constexpr int kMaxDecodeLocal = 16;     // local-branch chunks a decode step supports
 
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
   const int32_t* bt = a.block_table + (size_t)bi * a.max_chunks;
   const int L = a.seq_lens[bi];
   const int own = L > 0 ? (L - 1) / kChunk : 0;
-  const int n_cand = min(own, a.max_chunks);
+  const int n_cand = min(max(0, own + 1 - a.n_local), a.max_chunks);  // chunks before the local branch
   const int nc = max(0, min(n_cand, c_lo + R) - c_lo);
   for (int x = t; x < nc; x += kScanThreads) s_page[x] = bt[c_lo + x];
   // A page's summaries [h][d] are F 16-byte pieces.  When a page block is smaller than
@@ -363,13 +364,14 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
 }
 
 // ---------------------------------------------------------------------------
-// Attention: one warp per half chunk (32 keys) of the own chunk or of a Top-K slot,
-// all G heads sharing each K/V load.  Lanes own keys for Q.K (each reads its key row)
-// and output columns for P.V (V rows are read across the lanes); nothing is staged,
-// so many warps fit per SM.  Each warp writes its half's (max, sum, unnormalised
-// output) per head; the last CTA of the (sequence, KV head) combines the halves of
-// each chunk and fuses the chunks with the inter-chunk softmax of notes section 5.3
-// (own chunk at its exact log-mass).
+// Attention: one warp per half chunk (32 keys) of a local-branch chunk or of a Top-K
+// slot, all G heads sharing each K/V load.  Lanes own keys for Q.K (each reads its key
+// row) and output columns for P.V (V rows are read across the lanes); nothing is
+// staged, so many warps fit per SM.  Each warp writes its half's (max, sum,
+// unnormalised output) per head; the last CTA of the (sequence, KV head) combines the
+// halves of each chunk and fuses the chunks with the inter-chunk softmax of notes
+// section 5.3.  The local branch -- the own chunk, or with a sliding window the last
+// n_local chunks up to the new token -- enters as one term at its exact log-mass.
 constexpr int kAttWarps = 4;
 
 // Raw register types for one lane's share of a V row (CPL elements of T).
@@ -417,7 +419,7 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
   constexpr int EPP = 16 / (int)sizeof(T);     // elements per 16-byte piece
   constexpr int PPR = D / EPP;                 // pieces per key row
   __shared__ __align__(16) float qS[G][D];
-  __shared__ float s_w[G][2 * (kMaxTopK + 1)];  // fusion weight of each half chunk, per head
+  __shared__ float s_w[G][2 * (kMaxTopK + kMaxDecodeLocal)];  // fusion weight of each half chunk, per head
   __shared__ int s_last;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -426,7 +428,9 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
   const int gi = (blockIdx.x / ngrp) % a.g;
   const int bi = blockIdx.x / (ngrp * a.g);
   const int K = a.top_k;
-  const int n_items = 2 * (K + 1);             // item 2s + hf: slot s (0 own, s >= 1 Top-K s-1), half hf
+  const int NL = a.n_local;
+  // item 2s + hf: slot s < NL the local chunk own - s, slot s >= NL Top-K slot s - NL; half hf
+  const int n_items = 2 * (K + NL);
   const size_t part_stride = (size_t)G * (D + 2);
   float* part = a.part_att + ((size_t)bi * a.g + gi) * (size_t)n_items * part_stride;
   const int L = a.seq_lens[bi];
@@ -524,13 +528,16 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
       for (int x2 = 0; x2 < CPL; ++x2) dst[hh * (D + 2) + 2 + lane * CPL + x2] = o[hh][x2];
   };
 
-  // the own chunk does not depend on the selection: compute it before waiting
+  // the local branch does not depend on the selection: compute it before waiting
   const int own = L > 0 ? (L - 1) / kChunk : 0;
-  if (item < 2 && L > 0)
-    run_item(own, own < a.max_chunks ? a.block_table[(size_t)bi * a.max_chunks + own] : -1, L - own * kChunk);
+  if (item < 2 * NL && L > 0) {
+    const int c = own - (item >> 1);  // absent (c < 0) before the sequence's first chunk
+    run_item(c, c >= 0 && c < a.max_chunks ? a.block_table[(size_t)bi * a.max_chunks + c] : -1,
+             c == own ? L - own * kChunk : kChunk);
+  }
   pdl_wait_primary();
-  if (item >= 2 && item < n_items && L > 0) {
-    const size_t slot = ((size_t)bi * a.g + gi) * K + (item >> 1) - 1;
+  if (item >= 2 * NL && item < n_items && L > 0) {
+    const size_t slot = ((size_t)bi * a.g + gi) * K + (item >> 1) - NL;
     run_item(a.idx[slot], a.sel_page[slot], kChunk);
   }
 
@@ -546,25 +553,40 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
     if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
     return;
   }
-  // fusion weights, one warp per head: lane s handles slot s (3 rounds cover K + 1 <= 65 slots)
+  // fusion weights, one warp per head.  The local branch's halves (2 NL of them) are
+  // combined into (mL, lL), LSE_local = mL + log lL; then lane s handles Top-K slot s
+  // (2 rounds cover K <= 64 slots), its chunk's (m, l) combined from its halves.
   for (int hh = warp; hh < G; hh += kAttWarps) {
     const float* sc_row = a.ssel + ((size_t)bi * a.h + gi * G + hh) * K;
-    float lg[3], ms[3], ls[3], mh[3][2];
-    bool ok[3];
-    float M = -INFINITY;
+    float mloc = -INFINITY, lloc = 0.f;
+    for (int it = lane; it < 2 * NL; it += 32) {
+      const float* pp = part + (size_t)it * part_stride + hh * (D + 2);
+      const float mh = __ldcg(pp);
+      if (mh == -INFINITY) continue;
+      const float lh = __ldcg(pp + 1);
+      const float nm = fmaxf(mloc, mh);
+      lloc = lloc * expf(mloc - nm) + lh * expf(mh - nm);
+      mloc = nm;
+    }
+    const float mL = warp_max(mloc);
+    const float lL = warp_sum(mloc == -INFINITY ? 0.f : lloc * expf(mloc - mL));
+    const float lseL = mL + logf(lL);  // the own chunk always holds the new token: finite
+    float lg[2], ms[2], ls[2], mh[2][2];
+    bool ok[2];
+    float M = lseL;
 #pragma unroll
-    for (int rr = 0; rr < 3; ++rr) {
+    for (int rr = 0; rr < 2; ++rr) {
       const int sl = lane + 32 * rr;
       ok[rr] = false;
       lg[rr] = -INFINITY;
       ms[rr] = -INFINITY;
       ls[rr] = 0.f;
       mh[rr][0] = mh[rr][1] = -INFINITY;
-      if (sl < K + 1) {
+      if (sl < K) {
         float lh[2];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
-          const float* pp = part + (size_t)(2 * sl + h2) * part_stride + hh * (D + 2);
+          const float* pp = part + (size_t)(2 * (NL + sl) + h2) * part_stride + hh * (D + 2);
           mh[rr][h2] = __ldcg(pp);
           lh[h2] = mh[rr][h2] != -INFINITY ? __ldcg(pp + 1) : 0.f;
         }
@@ -574,7 +596,7 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2)
             if (mh[rr][h2] != -INFINITY) ls[rr] += lh[h2] * expf(mh[rr][h2] - ms[rr]);
-          lg[rr] = sl == 0 ? ms[rr] + logf(ls[rr]) : __ldcg(sc_row + sl - 1);
+          lg[rr] = __ldcg(sc_row + sl);
         }
       }
       M = fmaxf(M, lg[rr]);
@@ -582,18 +604,23 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
     M = warp_max(M);
     float z = 0.f;
 #pragma unroll
-    for (int rr = 0; rr < 3; ++rr) z += ok[rr] ? expf(lg[rr] - M) : 0.f;
-    const float Z = warp_sum(z);
+    for (int rr = 0; rr < 2; ++rr) z += ok[rr] ? expf(lg[rr] - M) : 0.f;
+    const float Z = warp_sum(z) + expf(lseL - M);
+    // local halves: exp(LSE_local - M)/Z * o/lL, i.e. exp(m_h - M)/Z * o_h per half
+    for (int it = lane; it < 2 * NL; it += 32) {
+      const float mhh = __ldcg(part + (size_t)it * part_stride + hh * (D + 2));
+      s_w[hh][it] = mhh == -INFINITY ? 0.f : expf(mhh - M) / Z;
+    }
 #pragma unroll
-    for (int rr = 0; rr < 3; ++rr) {
+    for (int rr = 0; rr < 2; ++rr) {
       const int sl = lane + 32 * rr;
-      if (sl < K + 1) {
-        // own: exp(LSE_own - M)/Z * o/l = exp(m - M)/Z * o ; selected: exp(shat - M)/(Z l) * o,
-        // with the chunk's (m, l, o) combined from its halves (o_h rescaled by exp(m_h - m))
-        const float wsl = !ok[rr] ? 0.f : (sl == 0 ? expf(ms[rr] - M) / Z : expf(lg[rr] - M) / (Z * ls[rr]));
+      if (sl < K) {
+        // selected: exp(shat - M)/(Z l) * o, with the chunk's (m, l, o) combined from its
+        // halves (o_h rescaled by exp(m_h - m))
+        const float wsl = !ok[rr] ? 0.f : expf(lg[rr] - M) / (Z * ls[rr]);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
-          s_w[hh][2 * sl + h2] = mh[rr][h2] == -INFINITY ? 0.f : wsl * expf(mh[rr][h2] - ms[rr]);
+          s_w[hh][2 * (NL + sl) + h2] = mh[rr][h2] == -INFINITY ? 0.f : wsl * expf(mh[rr][h2] - ms[rr]);
       }
     }
   }
@@ -657,7 +684,7 @@ static cudaError_t launch_decode(DecodeArgs a, cudaStream_t st) {
     }
     if (e != cudaSuccess) return e;
   }
-  a.att_ctas = (2 * (a.top_k + 1) + kAttWarps - 1) / kAttWarps;
+  a.att_ctas = (2 * (a.top_k + a.n_local) + kAttWarps - 1) / kAttWarps;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(bg * a.att_ctas);
   cfg.blockDim = dim3(kAttWarps * 32);

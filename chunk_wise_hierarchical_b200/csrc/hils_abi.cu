@@ -15,6 +15,7 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 256;  // error word + reserved
 constexpr int kMaxWindow = 64 * 128;  // local branch of at most 128 chunks
+constexpr int kMaxDecodeLocal = 16;   // ... and of at most 16 in a decode step
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -88,7 +89,7 @@ DecodeLayout decode_layout(const hils_shape* s) {
   DecodeLayout L;
   size_t off = kHeader;
   L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
-  L.part_att = off; off = align_up(off + b * g * 2 * (K + 1) * G * (d + 2) * 4);  // half-chunk partials
+  L.part_att = off; off = align_up(off + b * g * 2 * (K + n_local(s)) * G * (d + 2) * 4);  // half-chunk partials
   L.scan_ticket = off; off = align_up(off + b * g * 4);
   L.att_ticket = off; off = align_up(off + b * g * 4);
   L.idx = off; off = align_up(off + b * g * K * 4);
@@ -329,7 +330,7 @@ hils_status hils_decode_ex(const hils_shape* s, const void* q, const void* k_pag
   if (summary_dtype != HILS_F32 && summary_dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
   if (summary_dtype == HILS_BF16 && s->dtype != HILS_BF16) return HILS_ERR_UNSUPPORTED;
   if (s->batch == 0) return HILS_OK;
-  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) != 1) return HILS_ERR_UNSUPPORTED;
+  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) > kMaxDecodeLocal) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
@@ -358,6 +359,7 @@ hils_status hils_decode_ex(const hils_shape* s, const void* q, const void* k_pag
   da.max_chunks = max_chunks; da.n_pages = n_pages; da.scale = eff_scale(s);
   da.bf16 = s->dtype == HILS_BF16;
   da.kbar_bf16 = summary_dtype == HILS_BF16;
+  da.n_local = n_local(s);
   return cuda_status(hils::run_decode(da, cs));
 }
 
@@ -413,7 +415,7 @@ StaticLayout static_decode_layout(const hils_shape* s) {
   L.scan_ticket = off; off += kStaticTicketSlots * 4;
   L.att_ticket = off; off += kStaticTicketSlots * 4;
   L.part_keys = off; off = align_up(off + b * g * nsplit * K * 8);
-  L.part_att = off; off = align_up(off + b * g * 2 * (K + 1) * G * (d + 2) * 4);  // half-chunk partials
+  L.part_att = off; off = align_up(off + b * g * 2 * (K + n_local(s)) * G * (d + 2) * 4);  // half-chunk partials
   L.idx = off; off = align_up(off + b * g * K * 4);
   L.sel_page = off; off = align_up(off + b * g * K * 4);
   L.ssel = off; off = align_up(off + b * h * K * 4);
@@ -453,7 +455,7 @@ hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   if (s->batch == 0) return HILS_OK;
-  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) != 1) return HILS_ERR_UNSUPPORTED;
+  if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) > kMaxDecodeLocal) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
@@ -480,6 +482,7 @@ hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k
   da.b = s->batch; da.h = s->heads_q; da.g = s->heads_kv; da.d = s->head_dim; da.top_k = s->top_k;
   da.max_chunks = max_chunks; da.n_pages = n_pages; da.scale = eff_scale(s);
   da.bf16 = s->dtype == HILS_BF16;
+  da.n_local = n_local(s);
   return cuda_status(hils::run_decode(da, (cudaStream_t)stream));
 }
 

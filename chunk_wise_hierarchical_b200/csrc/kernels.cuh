@@ -55,12 +55,13 @@ struct DecodeArgs {
   int32_t* sel_page;           // [b,g,K] page of each selected chunk
   float* ssel;                 // [b,h,K]
   unsigned long long* part_keys;  // [b,g,nsplit,K] per-range Top-K lists
-  float* part_att;             // [b,g,2(K+1),G,d+2]: per half chunk (max, sum, unnormalised output)
+  float* part_att;             // [b,g,2(K+n_local),G,d+2]: per half chunk (max, sum, unnormalised output)
   unsigned* scan_ticket;       // [b,g] (the scan uses entry (b, 0))
   unsigned* att_ticket;        // [b,g]
   unsigned* err;
   bool kbar_bf16;              // compact summary cache (bf16 models only)
   int b, h, g, d, top_k, max_chunks, n_pages;
+  int n_local;                 // local-branch chunks (1: own chunk; W / B for a window), <= 16
   int nsplit, range, att_ctas; // set by the launcher: scan ranges per sequence, chunks per range
   float scale;
   bool bf16;

@@ -36,6 +36,8 @@ CONFIGS = {
                          chunk=64, top_k=16, dtype="bf16", qkv_std=1.0, needles=8),
     "prefill_7b_gqa": dict(batch=1, heads_q=32, heads_kv=8, seq_len=32768, head_dim=128,
                            chunk=64, top_k=32, dtype="bf16", qkv_std=0.5, needles=8),
+    "train_16k": dict(batch=2, heads_q=16, heads_kv=16, seq_len=16384, head_dim=128,
+                      chunk=64, top_k=16, dtype="bf16", qkv_std=1.0, needles=0),
     "decode_32k": dict(batch=8, heads_q=16, heads_kv=16, seq_len=32768, head_dim=64,
                        chunk=64, top_k=16, dtype="bf16"),
     "decode_128k": dict(batch=8, heads_q=16, heads_kv=16, seq_len=131072, head_dim=64,

@@ -128,10 +128,10 @@ def test_summary_dtype_validation():
                               None, fake, 1 << 30, None) == 2
 
 
-def test_decode_with_a_window_is_not_yet_supported_by_the_decode_kernels():
+def test_decode_window_beyond_the_decode_limit_is_unsupported():
     lib = hils.lib()
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the call fails validation first
-    s = _shape(window=512, seq_len=4096)
+    s = _shape(window=64 * 17, seq_len=4096)
     assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 8, fake, 4, fake, None,
                            fake, 1 << 30, None) == 2
 

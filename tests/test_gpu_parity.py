@@ -196,7 +196,7 @@ def test_prefill_sliding_window_local_branch(kw):
 
 
 # --------------------------------------------------------------------------- decode
-def _gpu_decode(di, K):
+def _gpu_decode(di, K, window=0):
     P, g, B, d = di.k_pages.shape
     h = di.landmark_pages.shape[1]
     dev = "cuda"
@@ -205,7 +205,7 @@ def _gpu_decode(di, K):
     hb = torch.zeros((P, h), dtype=torch.float32, device=dev)
     hils.summarize_paged(kp, lp, torch.arange(P, dtype=torch.int32, device=dev), kbar, hb)
     out, idx = hils.decode(di.q.to(dev), kp, vp, kbar, hb, di.block_table.to(dev),
-                           di.seq_lens.to(dev), K, return_idx=True)
+                           di.seq_lens.to(dev), K, return_idx=True, window=window)
     torch.cuda.synchronize()
     return out, idx
 
@@ -226,14 +226,14 @@ def _slice_for_oracle(di, bsel, gsel):
     return q, kp, vp, lp, new_bt, [int(di.seq_lens[bsel])]
 
 
-def _check_decode(di, out, idx, K, pairs):
+def _check_decode(di, out, idx, K, pairs, window=0):
     bf16 = di.q.dtype == torch.bfloat16
     h = di.landmark_pages.shape[1]
     g = di.k_pages.shape[1]
     grp = h // g
     for (b, gsel) in pairs:
         q, kp, vp, lp, bt, sl = _slice_for_oracle(di, b, gsel)
-        ref = O.decode(q, kp, vp, lp, bt, sl, K)
+        ref = O.decode(q, kp, vp, lp, bt, sl, K, window=window or None)
         gi = idx[b, gsel].cpu().numpy()
         if sl[0] > 0:
             check_indices(gi[None], ref["key"][0][0][None], K)
@@ -241,11 +241,11 @@ def _check_decode(di, out, idx, K, pairs):
         want = ref["out"][0]
         if not np.array_equal(gi, ref["idx"][0, 0]):
             # near tie: compare with the oracle fused over the GPU's selection
-            want = _forced_decode(q, kp, vp, lp, bt, sl, gi)
+            want = _forced_decode(q, kp, vp, lp, bt, sl, gi, window=window)
         check_close(got, want, bf16)
 
 
-def _forced_decode(q, kp, vp, lp, bt, sl, gidx):
+def _forced_decode(q, kp, vp, lp, bt, sl, gidx, window=0):
     # rebuild a contiguous sequence from the slice and run the forced prefill oracle on its last row
     L = sl[0]
     pages = bt[0, : (L + 63) // 64]
@@ -256,7 +256,8 @@ def _forced_decode(q, kp, vp, lp, bt, sl, gidx):
     lm = lp64[pages[: L // 64]].transpose(1, 0, 2)[None]
     qq = np.zeros((1, grp, L, q.shape[-1]))
     qq[0, :, L - 1] = O._f64(q)[0]
-    res = O.forward(qq, k, v, lm, 64, len(gidx), rows=[L - 1], forced_idx=np.asarray(gidx)[None, None, None])
+    res = O.forward(qq, k, v, lm, 64, len(gidx), rows=[L - 1], forced_idx=np.asarray(gidx)[None, None, None],
+                    window=window or None)
     return res["out"][0, :, 0]
 
 
@@ -266,6 +267,16 @@ def test_decode_small_ragged(dtype):
                        seq_lens=[1, 64, 65, 300, 1000], spare_pages=3)
     out, idx = _gpu_decode(di, 4)
     _check_decode(di, out, idx, 4, [(b, g) for b in range(5) for g in range(2)])
+
+
+@pytest.mark.parametrize("dtype,window,G", [("bf16", 256, 1), ("f32", 192, 2), ("bf16", 512, 4)])
+def test_decode_sliding_window_local_branch(dtype, window, G):
+    """Decode with the chunk-aligned sliding-window local branch (notes sections 5.2-5.3):
+    the last window / 64 chunks up to the new token at their exact mass, candidates before."""
+    di = decode_inputs(6, 2 * G, 2, 0, 64, top_k=3, dtype=dtype, seed=8,
+                       seq_lens=[1, 64, 65, 300, 1000, 64 * 9 + 1], spare_pages=2)
+    out, idx = _gpu_decode(di, 3, window=window)
+    _check_decode(di, out, idx, 3, [(b, g) for b in range(6) for g in range(2)], window=window)
 
 
 def test_decode_gqa_d128():
