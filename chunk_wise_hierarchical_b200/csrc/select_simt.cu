@@ -141,21 +141,25 @@ __global__ void select_simt_kernel(SelectArgs a, int qt) {
 // Register variant for K <= 32: one thread per (query, head) -- thread t takes query
 // t / G and head t % G of its KV group, so a thread holds one d-row of q (shared
 // memory, padded rows) and computes its head's scores; the group's max comes from
-// shuffles over its G consecutive lanes.  Every lane of a group keeps the same sorted
-// list of the best KP keys in registers, plus its own head's score of each listed
-// chunk (shifted together with the keys).
+// shuffles over its G consecutive lanes.  Every lane of a group keeps the same list of
+// the best KP (key, chunk) pairs sorted by key in registers, plus its own head's score
+// of each listed chunk (shifted together with the keys).  Chunks arrive in increasing
+// index order, so a strict fp32 comparison of keys keeps the lower index first among
+// equal keys; non-finite keys never enter.
 template <int KP>
-__device__ __forceinline__ void sorted_insert2(unsigned long long (&L)[KP], float (&S)[KP], unsigned long long x,
+__device__ __forceinline__ void sorted_insert2(float (&L)[KP], int (&I)[KP], float (&S)[KP], float x, int c,
                                                float sx) {
 #pragma unroll
   for (int j = KP - 1; j > 0; --j) {
     const bool above_prev = x > L[j - 1];
     const bool above_here = x > L[j];
     L[j] = above_prev ? L[j - 1] : (above_here ? x : L[j]);
+    I[j] = above_prev ? I[j - 1] : (above_here ? c : I[j]);
     S[j] = above_prev ? S[j - 1] : (above_here ? sx : S[j]);
   }
   if (x > L[0]) {
     L[0] = x;
+    I[0] = c;
     S[0] = sx;
   }
 }
@@ -190,11 +194,12 @@ __global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
   }
   const int last_i = min(a.n - 1, qtile * QT + QT - 1);
   const int tile_cand = n_candidates(last_i, a.n_local, a.n_chunks);
-  unsigned long long L[KP];
-  float Sc[KP];
+  float L[KP], Sc[KP];
+  int I[KP];
 #pragma unroll
   for (int s = 0; s < KP; ++s) {
-    L[s] = 0ull;  // below every real key
+    L[s] = -INFINITY;  // below every candidate
+    I[s] = -1;
     Sc[s] = -INFINITY;
   }
   for (int c0 = 0; c0 < tile_cand; c0 += kSelCT) {
@@ -227,10 +232,7 @@ __global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
       float best = own;
 #pragma unroll
       for (int o = 1; o < G; o <<= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-      if (c < n_cand) {
-        const unsigned long long key = pack_key(best, c);
-        if (key > L[KP - 1]) sorted_insert2(L, Sc, key, own);
-      }
+      if (c < n_cand && best > L[KP - 1]) sorted_insert2(L, I, Sc, best, c, own);
     }
   }
   (void)lane;
@@ -240,9 +242,8 @@ __global__ void __launch_bounds__(128) select_group_kernel(SelectArgs a) {
 #pragma unroll
   for (int s = 0; s < KP; ++s) {
     if (s < K) {
-      const bool have = L[s] != 0ull;
-      if (hh == 0) idx_out[s] = have ? key_chunk(L[s]) : -1;
-      if (sc_out) sc_out[s] = have ? Sc[s] : -INFINITY;
+      if (hh == 0) idx_out[s] = I[s];
+      if (sc_out) sc_out[s] = I[s] >= 0 ? Sc[s] : -INFINITY;
     }
   }
 }

@@ -8,10 +8,13 @@
 // accumulate into one fp32 TMEM tile, S = Q.hi^T + Q.lo^T, which keeps the
 // score error near 2^-17 of |q||kbar| (well inside the 1e-3 tie band the
 // selection is judged by).  Each thread then owns one query row: it reads its
-// scores from TMEM eight columns at a time, adds H_c and keeps its best KP
-// packed keys (score, then lower chunk index) as a sorted list in registers;
-// a candidate that beats the list's last entry is inserted by one unrolled
-// compare-and-shift pass, so no step touches memory.
+// scores from TMEM 32 columns at a time, adds H_c and keeps its best KP
+// (score, chunk) pairs as a list sorted by score in registers.  Candidates
+// arrive in increasing chunk order, so a strict comparison on the fp32 score
+// alone already puts an earlier (lower-index) chunk first among equal scores:
+// a candidate enters only if its score is above the list's last, and is then
+// inserted by one unrolled compare-and-shift pass.  Non-finite scores never
+// enter (they are not candidates).
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_util.cuh"
@@ -22,17 +25,22 @@ namespace {
 constexpr int kSelThreads = 128;
 constexpr int kNc = 128;  // candidate chunks per tile
 
-// L is sorted in descending order; x > L[KP-1].  Shifts the tail down by one
-// and drops x into its place (keys are unique: they carry the chunk index).
+// S is sorted in descending order and x > S[KP-1]; entries of equal score stay
+// ahead of x (they came from lower chunk indices).  Shifts the tail down by one
+// and drops (x, c) into its place.
 template <int KP>
-__device__ __forceinline__ void sorted_insert(unsigned long long (&L)[KP], unsigned long long x) {
+__device__ __forceinline__ void sorted_insert_f(float (&S)[KP], int (&I)[KP], float x, int c) {
 #pragma unroll
   for (int j = KP - 1; j > 0; --j) {
-    const bool above_prev = x > L[j - 1];
-    const bool above_here = x > L[j];
-    L[j] = above_prev ? L[j - 1] : (above_here ? x : L[j]);
+    const bool above_prev = x > S[j - 1];
+    const bool above_here = x > S[j];
+    S[j] = above_prev ? S[j - 1] : (above_here ? x : S[j]);
+    I[j] = above_prev ? I[j - 1] : (above_here ? c : I[j]);
   }
-  if (x > L[0]) L[0] = x;
+  if (x > S[0]) {
+    S[0] = x;
+    I[0] = c;
+  }
 }
 }  // namespace
 
@@ -83,9 +91,13 @@ __global__ void __launch_bounds__(kSelThreads) select_tc_kernel(SelectArgs a) {
   const uint32_t tmem = tmem_base_s;
   const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
 
-  unsigned long long L[KP];
+  float S[KP];
+  int I[KP];
 #pragma unroll
-  for (int s = 0; s < KP; ++s) L[s] = 0;  // below every real key
+  for (int s = 0; s < KP; ++s) {
+    S[s] = -INFINITY;  // below every candidate
+    I[s] = -1;
+  }
   uint32_t phase = 0;
   bool failed = false;
   for (int c0 = 0; c0 < tile_cand; c0 += kNc) {
@@ -143,33 +155,32 @@ __global__ void __launch_bounds__(kSelThreads) select_tc_kernel(SelectArgs a) {
       break;
     }
     tc::fence_after_sync();
-    // this tile's candidates, eight TMEM columns at a time
+    // this tile's candidates, 32 TMEM columns at a time
 #pragma unroll 1
-    for (int cb = 0; cb < nc; cb += 8) {
-      float sv[8];
-      tc::tmem_ld8(tmem + cb + lane_off, sv);
+    for (int cb = 0; cb < nc; cb += 32) {
+      float sv[32];
+      tc::tmem_ld32(tmem + cb + lane_off, sv);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 32; ++u) {
         const int c = c0 + cb + u;
-        const unsigned long long key = pack_key(fmaf(sv[u], a.scale, s_h[cb + u]), c);
-        if (c < n_cand && key > L[KP - 1]) sorted_insert(L, key);
+        const float x = fmaf(sv[u], a.scale, s_h[cb + u]);
+        if (c < n_cand && x > S[KP - 1]) sorted_insert_f(S, I, x, c);
       }
     }
     tc::fence_before_sync();
     __syncthreads();  // TMEM and the summary tiles are reused by the next tile
     tc::fence_after_sync();
   }
-  // the list is already in descending key order; G = 1, so a key's score is the head's own score
+  // the list is already in descending order; G = 1, so the key is the head's own score
   if (active && !failed) {
     int32_t* idx_out = a.idx + ((size_t)hq * N + i) * K;
     float* sc_out = a.score ? a.score + ((size_t)hq * N + i) * K : nullptr;
 #pragma unroll
     for (int s = 0; s < KP; ++s) {
       if (s < K) {
-        const bool have = L[s] != 0;
-        idx_out[s] = have ? key_chunk(L[s]) : -1;
-        if (sc_out) sc_out[s] = have ? unorderable((uint32_t)(L[s] >> 32)) : -INFINITY;
+        idx_out[s] = I[s];
+        if (sc_out) sc_out[s] = I[s] >= 0 ? S[s] : -INFINITY;
       }
     }
   }
