@@ -19,6 +19,9 @@ from ._abi import (  # noqa: F401
     OP_BACKWARD,
     decode,
     decode_static,
+    device_status,
+    set_wait_limit,
+    DEFAULT_WAIT_LIMIT,
     select,
     summarize,
     summarize_paged,

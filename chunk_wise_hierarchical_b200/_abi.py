@@ -70,6 +70,7 @@ def lib():
         "hils_decode_ex": (i32, [S, _P, _P, _P, _P, i32, _P, _P, i32, _P, i32, _P, _P, _P, sz, _P]),
         "hils_decode_static": (i32, [S, _P, _P, _P, _P, _P, _P, i32, _P, i32, _P, _P, _P, _P]),
         "hils_device_status": (i32, [_P, _P]),
+        "hils_set_wait_limit": (ctypes.c_uint32, [ctypes.c_uint32]),
         "hils_backward": (i32, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
     }
     for name, (res, args) in sig.items():
@@ -81,8 +82,21 @@ def lib():
 
 
 EXPORTED = ["hils_abi_version", "hils_attend", "hils_attend_selected", "hils_backward", "hils_decode",
-            "hils_decode_ex", "hils_decode_static", "hils_device_status", "hils_summarize_paged_ex", "hils_select", "hils_status_string", "hils_summarize",
-            "hils_summarize_paged", "hils_workspace_size"]
+            "hils_decode_ex", "hils_decode_static", "hils_device_status", "hils_summarize_paged_ex", "hils_select", "hils_set_wait_limit",
+            "hils_status_string", "hils_summarize", "hils_summarize_paged", "hils_workspace_size"]
+
+DEFAULT_WAIT_LIMIT = 1 << 26  # HILS_DEFAULT_WAIT_LIMIT
+
+
+def set_wait_limit(polls: int) -> int:
+    """Polls of an ordinary bounded device wait before a tensor-core kernel gives up
+    (process-wide; 0 gives up at once).  Returns the previous limit."""
+    return int(lib().hils_set_wait_limit(int(polls)))
+
+
+def device_status(ws, stream=None) -> int:
+    """Reads and clears the error word of a workspace (hils_device_status)."""
+    return int(lib().hils_device_status(_ptr(ws), _stream(stream)))
 
 
 def _dt(t: torch.Tensor) -> int:
@@ -158,13 +172,15 @@ def summarize_paged(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages, 
                                          _ptr(hbias_pages), _stream(stream)), "hils_summarize_paged_ex")
 
 
-def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True, window=0):
-    """topk_idx [b,g,N,K] int32 and (optionally) topk_score [b,h,N,K] fp32."""
+def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores=True, window=0, ws=None):
+    """topk_idx [b,g,N,K] int32 and (optionally) topk_score [b,h,N,K] fp32; `ws`, if
+    given, is the workspace whose error word the kernels report into."""
     b, h, n, d = q.shape
     sh = make_shape(b, h, heads_kv, d, n, top_k, _dt(q), scale=scale or 0.0, window=window)
     idx = torch.empty((b, heads_kv, n, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, h, n, top_k), dtype=torch.float32, device=q.device) if with_scores else None
-    ws = new_workspace(sh, OP_SELECT, q.device)
+    if ws is None:
+        ws = new_workspace(sh, OP_SELECT, q.device)
     _check(lib().hils_select(ctypes.byref(sh), _ptr(q), _ptr(kbar), _ptr(hbias), _ptr(idx), _ptr(sc),
                              _ptr(ws), ws.numel(), _stream(stream)), "hils_select")
     return idx, sc

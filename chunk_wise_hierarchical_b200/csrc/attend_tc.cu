@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   auto stage_ptr = [&](int s) -> unsigned char* { return sm + L.stage + s * C::kStageStride; };
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     const uint32_t b = tc::smem_u32(bar);
-    for (uint32_t it = 0; it < (1u << 26); ++it) {
+    for (uint32_t it = 0; it < a.poll; ++it) {
       if (tc::mbar_test(b, parity)) return true;
       if ((it & 1023u) == 1023u && s_abort) return false;
     }
@@ -324,14 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     // ======================= producer: Q rows (cp.async gather) + K chunk (TMA) =======================
     // The Q rows are written through the generic proxy: each lane waits for its own
     // copies, fences them for the tensor core (async proxy), then arrives.  With two
-    // stages one item's copies stay in flight while the next item is issued.
+    // stages one item's copies stay in flight while the next item is issued.  Every
+    // decision to stop is taken by the whole warp (the counts below stay warp-uniform).
+    int issued = 0, published = 0;
     auto publish = [&](int j) {  // item j's copies are complete and fenced
       tc::fence_async_smem();
       mbar_arrive(tc::smem_u32(&bar_full_qk[j % NS]));
+      ++published;
     };
     for (int i = 0; i < n_items; ++i) {
       const int s = i % NS;
-      if (i >= NS && !wait(&bar_sfull[(i - NS) % NP], (uint32_t)(((i - NS) / NP) & 1))) break;
+      if (i >= NS && !__all_sync(0xffffffffu, wait(&bar_sfull[(i - NS) % NP], (uint32_t)(((i - NS) / NP) & 1))))
+        break;
       int c, t0, n_rows;
       bool own;
       item_rows(s_items[i], c, own, t0, n_rows);
@@ -353,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
           tc::cp_async16(sA + (uint32_t)(ch >> 3) * 16384u + tc::sw128_chunk(t, ch & 7), src + ch * 8);
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
+      ++issued;
       if constexpr (NS == 1) {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         publish(i);
@@ -366,12 +371,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
           publish(i);
         }
       }
-      if (s_abort) break;
+      if (__any_sync(0xffffffffu, s_abort != 0)) break;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+    // On the way out (normal or aborted) no copy may still be writing shared memory when the
+    // CTA ends: items issued but not yet published are published now, so that their barrier
+    // phases complete once the K tiles land, and lane 0 waits (drain bound) for the newest
+    // phase of every stage used.
+    while (published < issued) publish(published);
+    if (lane == 0)
+      for (int j = max(0, issued - NS); j < issued; ++j)
+        tc::mbar_wait(tc::smem_u32(&bar_full_qk[j % NS]), (uint32_t)((j / NS) & 1), kDrainPolls);
   } else if (warp == 1) {
     // ======================= producer: V chunk (TMA) =======================
     if (lane == 0) {
+      int issued = 0;
       for (int i = 0; i < n_items; ++i) {
         const int s = i % NS;
         // P.V of item i - NS, the last reader of this stage's V, must have completed
@@ -382,7 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         tc::mbar_arrive_expect_tx(full, C::kStageV);
 #pragma unroll
         for (int x = 0; x < D / 64; ++x) tc::tma_load_3d(sV + x * 8192u, &a.tmap_v, x * 64, c * kChunk, bi * a.g + gi, full);
+        ++issued;
+        if (s_abort) break;
       }
+      // every issued copy has landed before the CTA's shared memory is released
+      for (int j = max(0, issued - NS); j < issued; ++j)
+        tc::mbar_wait(tc::smem_u32(&bar_full_v[j % NS]), (uint32_t)((j / NS) & 1), kDrainPolls);
     }
   } else if (warp == 2) {
     // ======================= MMA issuer =======================
@@ -438,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         }
         if (progressed) {
           idle = 0;
-        } else if (++idle >= (1u << 26) || ((idle & 1023u) == 1023u && s_abort)) {
+        } else if (++idle >= a.poll || ((idle & 1023u) == 1023u && s_abort)) {
           if (!s_abort) {
             set_error(a.err, kErrTimeout);
             s_abort = 1;
@@ -446,6 +465,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
           break;
         }
       }
+      // every MMA issued has completed before the tensor memory is released: MMAs complete
+      // in issue order, and only this thread commits, so the last commit of each ring is
+      // the newest phase of its barrier
+      if (next_s > 0)
+        tc::mbar_wait(tc::smem_u32(&bar_sfull[(next_s - 1) % NP]), (uint32_t)(((next_s - 1) / NP) & 1), kDrainPolls);
+      if (next_pv > 0)
+        tc::mbar_wait(tc::smem_u32(&bar_ofull[(next_pv - 1) % NO]), (uint32_t)(((next_pv - 1) / NO) & 1), kDrainPolls);
     }
   } else if (warp >= 4 && warp < 12) {
     // ======================= softmax (two warpgroups, alternating items) =======================
@@ -511,7 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         named_bar(1, 256);  // every row's (M, 1/Z') is final once the own items are done
         synced_own = true;
       }
-      if (!wait(&bar_sfull[b], (uint32_t)((i / NP) & 1))) break;
+      // the warp leaves together (the tensor-memory loads below are warp-collective)
+      if (!__all_sync(0xffffffffu, wait(&bar_sfull[b], (uint32_t)((i / NP) & 1)))) break;
       tc::fence_after_sync();
       const bool row_ok = t < n_rows;
       if (wq * 32 < n_rows) {

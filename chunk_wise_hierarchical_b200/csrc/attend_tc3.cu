@@ -53,7 +53,6 @@ namespace {
 constexpr int kThreads3 = 512;
 constexpr float kLog2e3 = 1.4426950408889634f;
 constexpr uint32_t kOwnFlag3 = 0x80000000u;
-constexpr uint32_t kPoll = 1u << 26;  // bound of every mbarrier wait
 
 struct Cfg3 {
   static constexpr int D = 64;
@@ -387,7 +386,7 @@ __global__ void __launch_bounds__(kThreads3, 1) attend_tc3_kernel(const __grid_c
   auto stage_u32 = [&](int s) -> uint32_t { return tc::smem_u32(sm + L.stage + s * C::kStage); };
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     const uint32_t b = tc::smem_u32(bar);
-    for (uint32_t it = 0; it < kPoll; ++it) {
+    for (uint32_t it = 0; it < a.poll; ++it) {
       if (tc::mbar_test(b, parity)) return true;
       if ((it & 1023u) == 1023u && s_abort) return false;
     }
@@ -423,7 +422,7 @@ __global__ void __launch_bounds__(kThreads3, 1) attend_tc3_kernel(const __grid_c
       // on the way out (normal or aborted), every issued copy has landed before the CTA's
       // shared memory is released: wait (bounded) for the last phase of each used stage
       for (int j = max(0, issued - NS); j < issued; ++j)
-        tc::mbar_wait(tc::smem_u32(&bar_kv[j % NS]), (uint32_t)((j / NS) & 1), kPoll);
+        tc::mbar_wait(tc::smem_u32(&bar_kv[j % NS]), (uint32_t)((j / NS) & 1), kDrainPolls);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
@@ -480,8 +479,8 @@ __global__ void __launch_bounds__(kThreads3, 1) attend_tc3_kernel(const __grid_c
       // every MMA issued has completed before the tensor memory is released: MMAs complete
       // in issue order, and only this thread commits, so the last commit of each ring is
       // the newest phase of its barrier
-      if (next_s > 0) tc::mbar_wait(tc::smem_u32(&bar_sfull[(next_s - 1) % NP]), (uint32_t)(((next_s - 1) / NP) & 1), kPoll);
-      if (next_pv > 0) tc::mbar_wait(tc::smem_u32(&bar_ofull[(next_pv - 1) % NO]), (uint32_t)(((next_pv - 1) / NO) & 1), kPoll);
+      if (next_s > 0) tc::mbar_wait(tc::smem_u32(&bar_sfull[(next_s - 1) % NP]), (uint32_t)(((next_s - 1) / NP) & 1), kDrainPolls);
+      if (next_pv > 0) tc::mbar_wait(tc::smem_u32(&bar_ofull[(next_pv - 1) % NO]), (uint32_t)(((next_pv - 1) / NO) & 1), kDrainPolls);
     }
   }
   } else if (warp >= 4 && warp < 12) {
@@ -573,7 +572,8 @@ __global__ void __launch_bounds__(kThreads3, 1) attend_tc3_kernel(const __grid_c
         bar_sync(1, 256);  // every row's (M, 1/Z') is final once the own items are done
         synced_own = true;
       }
-      if (!wait(&bar_sfull[b], (uint32_t)((i / NP) & 1))) break;
+      // the warp leaves together (the tensor-memory loads below are warp-collective)
+      if (!__all_sync(0xffffffffu, wait(&bar_sfull[b], (uint32_t)((i / NP) & 1)))) break;
       tc::fence_after_sync();
       // S(i) is done, so Q slot i % NQ is free again: store the rows of item i + 2
       const bool refill = i + 2 < n_items;

@@ -16,6 +16,11 @@ constexpr int kMaxTopK = 64;
 constexpr unsigned kErrBadPage = 1u;
 constexpr unsigned kErrTimeout = 2u;
 
+// Polls of the waits that drain an abort path (copies and MMAs already issued
+// finish before shared and tensor memory are released).  They use this bound
+// whatever limit the caller set for ordinary waits.
+constexpr uint32_t kDrainPolls = HILS_DEFAULT_WAIT_LIMIT;
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 

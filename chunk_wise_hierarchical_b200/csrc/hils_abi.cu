@@ -4,6 +4,7 @@
 // (except hils_device_status).
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/hils.h"
@@ -11,6 +12,9 @@
 #include "kernels.cuh"
 
 namespace {
+
+// Polls of an ordinary bounded wait in the tensor-core kernels (hils_set_wait_limit).
+std::atomic<uint32_t> g_wait_limit{HILS_DEFAULT_WAIT_LIMIT};
 
 constexpr size_t kAlign = 256;
 constexpr size_t kHeader = 256;  // error word + reserved
@@ -116,6 +120,7 @@ cudaError_t run_prefill_attention(const hils_shape* s, const void* q, const void
     ta.idx = idx; ta.ssel = ssel; ta.out = static_cast<__nv_bfloat16*>(out); ta.lse = lse; ta.err = err;
     ta.b = s->batch; ta.h = s->heads_q; ta.g = s->heads_kv; ta.n = s->seq_len; ta.top_k = s->top_k;
     ta.scale = eff_scale(s);
+    ta.poll = g_wait_limit.load();
     return hils::run_attend_tc(ta, s->head_dim, cs);
   }
   hils::AttendRowsArgs ar{};
@@ -144,7 +149,9 @@ const char* hils_status_string(int status) {
   return "unknown status";
 }
 
-int32_t hils_abi_version(void) { return 2; }
+int32_t hils_abi_version(void) { return 3; }
+
+uint32_t hils_set_wait_limit(uint32_t polls) { return g_wait_limit.exchange(polls); }
 
 hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) {
   if (!bytes) return HILS_ERR_INVALID_ARG;
@@ -205,7 +212,11 @@ hils_status hils_summarize_paged_ex(const hils_shape* s, const void* k_pages, co
 
 // Scores + Top-K: the tensor-core kernel where it applies (bf16, G = 1), else SIMT.
 static cudaError_t run_select(const hils::SelectArgs& a, cudaStream_t st) {
-  if (hils::select_tc_supported(a.d, a.h / a.g, a.top_k, a.bf16)) return hils::run_select_tc(a, st);
+  if (hils::select_tc_supported(a.d, a.h / a.g, a.top_k, a.bf16)) {
+    hils::SelectArgs t = a;
+    t.poll = g_wait_limit.load();
+    return hils::run_select_tc(t, st);
+  }
   return hils::run_select_simt(a, st);
 }
 

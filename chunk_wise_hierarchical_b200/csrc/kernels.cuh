@@ -34,6 +34,7 @@ struct SelectArgs {
   int n_local;            // chunks in the local branch (1: own chunk; W / B for a window)
   float scale;
   bool bf16;
+  uint32_t poll;          // polls of a bounded wait before it gives up (tensor-core kernel)
 };
 cudaError_t run_select_simt(const SelectArgs& a, cudaStream_t st);
 // Tensor-core scores + Top-K (bf16, one query head per KV head).
@@ -106,6 +107,7 @@ struct alignas(64) TcAttendArgs {
   float scale;
   int qb;                      // queries per CTA (set by the launcher)
   int n_cand_max;              // N / chunk (set by the launcher)
+  uint32_t poll;               // polls of a bounded wait before it gives up
 };
 // Backward pass (bf16 inputs, fp32 gradients) for a forward's selection and row normaliser.
 struct BwdArgs {

@@ -145,15 +145,18 @@ __global__ void __launch_bounds__(kSelThreads) select_tc_kernel(SelectArgs a) {
       }
       tc::mma_commit(tc::smem_u32(&bar_mma));
     }
-    if (!tc::mbar_wait(tc::smem_u32(&bar_mma), phase)) {
+    if (!tc::mbar_wait(tc::smem_u32(&bar_mma), phase, a.poll)) {
       set_error(a.err, kErrTimeout);
       failed = true;
     }
-    phase ^= 1u;
     if (__syncthreads_or(failed)) {
+      // give up: the MMAs committed above may still be running; they finish (a wait with
+      // the drain bound) before the tensor memory is released below
+      tc::mbar_wait(tc::smem_u32(&bar_mma), phase, kDrainPolls);
       failed = true;
       break;
     }
+    phase ^= 1u;
     tc::fence_after_sync();
     // this tile's candidates, 32 TMEM columns at a time
 #pragma unroll 1

@@ -100,8 +100,27 @@ typedef struct {
 /* Static English text for a status code; never NULL. */
 HILS_API const char* hils_status_string(int status);
 
-/* ABI version, currently 2 (1 had no window field and no lse_out). */
+/* ABI version, currently 3 (1 had no window field and no lse_out; 2 had no
+ * hils_set_wait_limit). */
 HILS_API int32_t hils_abi_version(void);
+
+/* Default of hils_set_wait_limit: about a second or more of polling. */
+#define HILS_DEFAULT_WAIT_LIMIT (1u << 26)
+
+/*
+ * hils_set_wait_limit -- sets how many times an ordinary bounded wait of the
+ * tensor-core kernels (select, prefill attention) polls its mbarrier before the
+ * kernel gives up.  A kernel that gives up sets the timeout bit of the error
+ * word (hils_device_status then returns HILS_ERR_DEVICE_TIMEOUT), stops issuing
+ * work, waits for the copies and MMAs it has already issued (those drain waits
+ * always use HILS_DEFAULT_WAIT_LIMIT), releases its tensor memory and returns
+ * without writing its outputs; a later call on the same context runs normally.
+ * The limit is process-wide and read when a call launches its kernels (a CUDA
+ * graph keeps the value it was captured with).  0 makes every ordinary wait
+ * give up at its first poll: that is how the give-up path is exercised.
+ * Returns the previous limit.  Not a pages' operation; no error status.
+ */
+HILS_API uint32_t hils_set_wait_limit(uint32_t polls);
 
 /* Bytes of device workspace `op` needs for `shape`, written to *bytes.
  * HILS_OP_DECODE reads shape.seq_len as the largest cache length and

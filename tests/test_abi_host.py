@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings_and_version():
     lib = hils.lib()
-    assert lib.hils_abi_version() == 2
+    assert lib.hils_abi_version() == 3
     for code in range(7):
         assert lib.hils_status_string(code)
     assert lib.hils_status_string(99) == b"unknown status"
@@ -165,3 +165,18 @@ def test_backward_rejects_before_launch():
     assert lib.hils_backward(ctypes.byref(s16), *args, None, 0, None) == 3
     n = ctypes.c_size_t(0)
     assert lib.hils_workspace_size(ctypes.byref(s16), 4, ctypes.byref(n)) == 0 and n.value > 256
+
+
+def test_wait_limit_setter_returns_the_previous_limit():
+    """hils_set_wait_limit is host state only: the default is HILS_DEFAULT_WAIT_LIMIT
+    (parsed from the header) and each call returns the limit it replaces."""
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hils.h")).read()
+    m = re.search(r"#define HILS_DEFAULT_WAIT_LIMIT \(1u << (\d+)\)", hdr)
+    assert m and hils.DEFAULT_WAIT_LIMIT == 1 << int(m.group(1))
+    prev = hils.set_wait_limit(12345)
+    try:
+        assert prev == hils.DEFAULT_WAIT_LIMIT
+        assert hils.set_wait_limit(0) == 12345
+    finally:
+        hils.set_wait_limit(prev)
+    assert hils.set_wait_limit(prev) == prev
