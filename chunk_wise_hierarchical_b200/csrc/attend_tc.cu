@@ -749,6 +749,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // A [b*g][N][D] bf16 tensor as a rank-3 map with 64 x 64 boxes in the 128-byte
 // swizzle of the MMA operand tiles; rows past N read as zeros.
 static bool encode_kv_map(CUtensorMap* m, const void* base, int D, int N, int bg) {
+  return encode_kv_tensor_map(m, base, D, N, bg);
+}
+bool encode_kv_tensor_map(CUtensorMap* m, const void* base, int D, int N, int bg) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)bg};

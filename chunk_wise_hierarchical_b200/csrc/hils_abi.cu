@@ -51,8 +51,26 @@ float eff_scale(const hils_shape* s) {
   return s->scale == 0.f ? 1.0f / std::sqrt((float)s->head_dim) : s->scale;
 }
 
+// Whether prefill attention takes the chunk-major tensor-core path for this shape (its
+// scratch is then part of the workspace); the kernel's register check comes at launch.
+bool cm_applies(const hils_shape* s) {
+  if (s->dtype != HILS_BF16 || s->heads_kv <= 0) return false;
+  const int G = s->heads_q / s->heads_kv;
+  if (!hils::cm_shape_supported(s->head_dim, G, s->top_k, s->seq_len, n_local(s))) return false;
+  const hils::CmScratch S = hils::cm_scratch(s->batch, s->heads_q, s->heads_kv, s->seq_len, s->head_dim,
+                                             s->top_k, n_local(s));
+  // partial rows and selection indices are 32-bit
+  return ((size_t)S.n_lt + S.max_sel) * 128 < (1ull << 31) &&
+         (size_t)s->batch * s->heads_kv * s->seq_len * s->top_k < (1ull << 31) &&
+         (size_t)s->batch * s->heads_q * s->seq_len < (1ull << 31);
+}
+size_t cm_bytes(const hils_shape* s) {
+  if (!cm_applies(s)) return 0;
+  return hils::cm_scratch(s->batch, s->heads_q, s->heads_kv, s->seq_len, s->head_dim, s->top_k, n_local(s)).total;
+}
+
 struct AttendLayout {
-  size_t kbar, hbias, idx, ssel, total;
+  size_t kbar, hbias, idx, ssel, cm, total;
 };
 AttendLayout attend_layout(const hils_shape* s) {
   const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, n = s->seq_len, d = s->head_dim;
@@ -63,6 +81,7 @@ AttendLayout attend_layout(const hils_shape* s) {
   L.hbias = off; off = align_up(off + b * h * C * 4);
   L.idx = off; off = align_up(off + b * g * n * K * 4);
   L.ssel = off; off = align_up(off + b * h * n * K * 4);
+  L.cm = off; off = align_up(off + cm_bytes(s));
   L.total = off;
   return L;
 }
@@ -105,13 +124,44 @@ DecodeLayout decode_layout(const hils_shape* s) {
 
 hils_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA; }
 
-// Prefill attention + fusion for a selection: the tcgen05 kernel for bf16
-// inputs when its shared-memory plan fits the shape, else the row kernel.
+// Prefill attention + fusion for a selection: the chunk-major tcgen05 path for bf16
+// inputs (scratch at `cm_ws`, 256-byte aligned), else the row-owner tcgen05 kernels
+// where they fit the shape, else the row kernel.
 cudaError_t run_prefill_attention(const hils_shape* s, const void* q, const void* k, const void* v,
                                   const int32_t* idx, const float* ssel, void* out, float* lse,
-                                  unsigned* err, cudaStream_t cs) {
+                                  unsigned* err, void* cm_ws, cudaStream_t cs) {
   const bool bf16 = s->dtype == HILS_BF16;
   const int G = s->heads_q / s->heads_kv;
+  // d = 64 with the own-chunk branch stays on the row-owner kernel, measured faster there;
+  // every other bf16 shape the chunk-major path covers takes it
+  const bool row_owner_d64 = bf16 && n_local(s) == 1 && s->head_dim == 64 &&
+                             hils::attend_tc3_supported(64, G, s->top_k, s->seq_len);
+  if (!row_owner_d64 && cm_ws && cm_applies(s) && hils::cm_kernel_ready(s->head_dim, G)) {
+    const hils::CmScratch S = hils::cm_scratch(s->batch, s->heads_q, s->heads_kv, s->seq_len, s->head_dim,
+                                               s->top_k, n_local(s));
+    char* w = static_cast<char*>(cm_ws);
+    hils::CmArgs a{};
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.idx = idx; a.ssel = ssel; a.out = static_cast<__nv_bfloat16*>(out); a.lse = lse; a.err = err;
+    a.cnt = reinterpret_cast<int*>(w + S.cnt);
+    a.cur = reinterpret_cast<int*>(w + S.cur);
+    a.toff = reinterpret_cast<int*>(w + S.toff);
+    a.n_sel = reinterpret_cast<int*>(w + S.n_sel);
+    a.abort_flag = reinterpret_cast<int*>(w + S.abort_flag);
+    a.desc = reinterpret_cast<int4*>(w + S.desc);
+    a.ent_q = reinterpret_cast<int*>(w + S.ent_q);
+    a.pos = reinterpret_cast<int*>(w + S.pos);
+    a.part = reinterpret_cast<__nv_bfloat16*>(w + S.part);
+    a.plse = reinterpret_cast<float*>(w + S.plse);
+    a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
+    a.top_k = s->top_k; a.n_local = n_local(s);
+    a.c_sel = S.c_sel; a.c_all = S.c_all; a.tl = S.tl; a.n_lt = S.n_lt; a.max_sel = S.max_sel;
+    a.scale = eff_scale(s);
+    a.poll = g_wait_limit.load();
+    return hils::run_attend_cm(a, cs);
+  }
   if (bf16 && n_local(s) == 1 && hils::attend_tc_supported(s->head_dim, G, s->top_k, s->seq_len)) {
     hils::TcAttendArgs ta{};
     ta.q = static_cast<const __nv_bfloat16*>(q);
@@ -161,7 +211,7 @@ hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) 
     case HILS_OP_SELECT: *bytes = kHeader; return HILS_OK;
     case HILS_OP_ATTEND: *bytes = attend_layout(s).total; return HILS_OK;
     case HILS_OP_DECODE: *bytes = decode_layout(s).total; return HILS_OK;
-    case HILS_OP_ATTEND_SELECTED: *bytes = kHeader; return HILS_OK;
+    case HILS_OP_ATTEND_SELECTED: *bytes = kHeader + cm_bytes(s); return HILS_OK;
     case HILS_OP_BACKWARD: *bytes = backward_layout(s).total; return HILS_OK;
   }
   return HILS_ERR_INVALID_ARG;
@@ -275,8 +325,8 @@ hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const
     se.err = reinterpret_cast<unsigned*>(w);
     if (run_select(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
   }
-  return cuda_status(
-      run_prefill_attention(s, q, k, v, idx, ssel, out, lse_out, reinterpret_cast<unsigned*>(w), cs));
+  return cuda_status(run_prefill_attention(s, q, k, v, idx, ssel, out, lse_out, reinterpret_cast<unsigned*>(w),
+                                           L.cm != L.total ? w + L.cm : nullptr, cs));
 }
 
 hils_status hils_attend_selected(const hils_shape* s, const void* q, const void* k, const void* v,
@@ -287,9 +337,12 @@ hils_status hils_attend_selected(const hils_shape* s, const void* q, const void*
   if ((size_t)s->batch * s->seq_len == 0) return HILS_OK;
   if (!q || !k || !v || !out || (s->top_k > 0 && (!topk_idx || !topk_score))) return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HILS_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  const size_t cmb = cm_bytes(s);
+  if (!ws || ws_bytes < kHeader + cmb || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  char* w = static_cast<char*>(ws);
   return cuda_status(run_prefill_attention(s, q, k, v, topk_idx, topk_score, out, lse_out,
-                                           reinterpret_cast<unsigned*>(ws), (cudaStream_t)stream));
+                                           reinterpret_cast<unsigned*>(ws), cmb ? w + kHeader : nullptr,
+                                           (cudaStream_t)stream));
 }
 
 hils_status hils_backward(const hils_shape* s, const void* q, const void* k, const void* v,

@@ -133,6 +133,52 @@ struct BwdArgs {
 };
 cudaError_t run_backward(const BwdArgs& a, cudaStream_t st);
 
+// Chunk-major prefill attention (bf16, d = 64 or 128, G in {1, 2, 4, 8}): every
+// (query, selected chunk) pair of the whole sequence is bucketed by chunk into full
+// 128-row tiles; each tile's normalised chunk output is stored as a bf16 partial and
+// a fusion pass combines a row's partials with the inter-chunk softmax.
+struct alignas(64) CmArgs {
+  CUtensorMap tmap_k;          // K as [b*g][N][d], 64x64 boxes, 128B swizzle
+  CUtensorMap tmap_v;          // V, likewise
+  const __nv_bfloat16* q;      // [b,h,N,d]
+  const __nv_bfloat16* k;      // [b,g,N,d]
+  const __nv_bfloat16* v;
+  const int32_t* idx;          // [b,g,N,K]
+  const float* ssel;           // [b,h,N,K]
+  __nv_bfloat16* out;          // [b,h,N,d]
+  float* lse;                  // [b,h,N] log Zhat, or nullptr
+  unsigned* err;
+  // workspace (see cm_scratch_bytes)
+  int* cnt;                    // [b*g*c_sel] selections per (sequence, KV head, chunk)
+  int* cur;                    // [b*g*c_sel] scatter cursors
+  int* toff;                   // [b*g*c_sel + 1] first selected tile of each bucket
+  int* n_sel;                  // number of selected tiles
+  int* abort_flag;             // set when the tile kernel gave up (the fusion then writes nothing)
+  int4* desc;                  // per selected tile: (b*g + KV head, chunk, first entry, rows)
+  int* ent_q;                  // per selected tile: 128 / G entries, the Q row (of [b*h*N]) of the group's first head, -1 padding
+  int* pos;                    // [b,g,N,K] partial row of each selection (head 0 of the group), -1 if none
+  __nv_bfloat16* part;         // [tiles][128][d] normalised chunk outputs
+  float* plse;                 // [local tiles][128] log-mass of each local-branch chunk
+  int b, h, g, n, d, top_k, n_local;
+  int c_sel;                   // N / B: complete chunks (selectable)
+  int c_all;                   // ceil(N / B): chunks with a local bucket
+  int tl;                      // tiles per local bucket
+  int n_lt;                    // local tiles = b * g * c_all * tl
+  int max_sel;                 // capacity of the selected-tile arrays
+  float scale;
+  uint32_t poll;               // polls of a bounded wait before it gives up
+};
+bool cm_shape_supported(int d, int G, int K, int N, int n_local);
+bool cm_kernel_ready(int d, int G);  // compiled to the register budget its warp roles assume
+// Bytes of scratch the chunk-major path needs, and its offsets from a 256-byte aligned base.
+struct CmScratch {
+  size_t cnt, cur, toff, n_sel, abort_flag, desc, ent_q, pos, part, plse, total;
+  int c_sel, c_all, tl, n_lt, max_sel;
+};
+CmScratch cm_scratch(int b, int h, int g, int n, int d, int K, int n_local);
+cudaError_t run_attend_cm(CmArgs a, cudaStream_t st);
+bool encode_kv_tensor_map(CUtensorMap* m, const void* base, int D, int N, int bg);
+
 bool attend_tc_supported(int d, int G, int K, int N);
 cudaError_t run_attend_tc(const TcAttendArgs& a, int d, cudaStream_t st);
 // Head dim 64: Q rows in tensor memory, conflict-free accumulation order (tensor maps set).

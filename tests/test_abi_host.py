@@ -44,11 +44,21 @@ def _shape(**kw):
 
 
 def test_workspace_sizes():
-    s = _shape()
+    # fp32 inputs: summaries, selection and scores only
+    s = _shape(dtype=0)
     n = _abi.workspace_size(s, _abi.OP_ATTEND)
     C = 1000 // 64
     need = 2 * 8 * C * 64 * 4 + 2 * 8 * C * 4 + 2 * 2 * 1000 * 16 * 4 + 2 * 8 * 1000 * 16 * 4
     assert need <= n <= need + 6 * 256
+    assert _abi.workspace_size(s, _abi.OP_ATTEND_SELECTED) == 256
+    # bf16 inputs: also the chunk-major scratch, at least one d-wide bf16 partial per
+    # (query, head, slot) and per local-branch row, plus their positions
+    s = _shape()
+    partials = (2 * 8 * 1000 * 16 + 2 * 8 * 1000) * 64 * 2 + 2 * 2 * 1000 * 16 * 4
+    n = _abi.workspace_size(s, _abi.OP_ATTEND)
+    assert need + partials <= n <= 2 * (need + partials)
+    m = _abi.workspace_size(s, _abi.OP_ATTEND_SELECTED)
+    assert 256 + partials <= m <= n - need + 256
     assert _abi.workspace_size(s, _abi.OP_SELECT) == 256
     assert _abi.workspace_size(s, _abi.OP_DECODE) >= 2 * 2 * 16 * 8
 
