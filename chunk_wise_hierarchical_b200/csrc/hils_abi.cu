@@ -69,8 +69,22 @@ size_t cm_bytes(const hils_shape* s) {
   return hils::cm_scratch(s->batch, s->heads_q, s->heads_kv, s->seq_len, s->head_dim, s->top_k, n_local(s)).total;
 }
 
+// Whether selection takes the grouped tensor-core path (its split summaries are then
+// part of the workspace): bf16, G in {2, 4, 8}, at least one full tile of chunks and of
+// queries.
+bool gtc_applies(const hils_shape* s) {
+  if (s->dtype != HILS_BF16 || s->heads_kv <= 0) return false;
+  const int G = s->heads_q / s->heads_kv;
+  return hils::select_gtc_supported(s->head_dim, G, s->top_k, true) && s->seq_len / s->chunk >= 64 &&
+         s->seq_len >= 128;
+}
+size_t gtc_bytes(const hils_shape* s) {
+  if (!gtc_applies(s)) return 0;
+  return 2 * align_up(hils::gtc_split_bytes(s->batch, s->heads_q, s->seq_len / s->chunk, s->head_dim));
+}
+
 struct AttendLayout {
-  size_t kbar, hbias, idx, ssel, cm, total;
+  size_t kbar, hbias, idx, ssel, gtc, cm, total;
 };
 AttendLayout attend_layout(const hils_shape* s) {
   const size_t b = s->batch, h = s->heads_q, g = s->heads_kv, n = s->seq_len, d = s->head_dim;
@@ -81,6 +95,7 @@ AttendLayout attend_layout(const hils_shape* s) {
   L.hbias = off; off = align_up(off + b * h * C * 4);
   L.idx = off; off = align_up(off + b * g * n * K * 4);
   L.ssel = off; off = align_up(off + b * h * n * K * 4);
+  L.gtc = off; off = align_up(off + gtc_bytes(s));
   L.cm = off; off = align_up(off + cm_bytes(s));
   L.total = off;
   return L;
@@ -208,7 +223,7 @@ hils_status hils_workspace_size(const hils_shape* s, int32_t op, size_t* bytes) 
   hils_status st = check_shape(s, true);
   if (st != HILS_OK) return st;
   switch (op) {
-    case HILS_OP_SELECT: *bytes = kHeader; return HILS_OK;
+    case HILS_OP_SELECT: *bytes = kHeader + gtc_bytes(s); return HILS_OK;
     case HILS_OP_ATTEND: *bytes = attend_layout(s).total; return HILS_OK;
     case HILS_OP_DECODE: *bytes = decode_layout(s).total; return HILS_OK;
     case HILS_OP_ATTEND_SELECTED: *bytes = kHeader + cm_bytes(s); return HILS_OK;
@@ -261,11 +276,24 @@ hils_status hils_summarize_paged_ex(const hils_shape* s, const void* k_pages, co
 }
 
 // Scores + Top-K: the tensor-core kernel where it applies (bf16, G = 1), else SIMT.
-static cudaError_t run_select(const hils::SelectArgs& a, cudaStream_t st) {
+// gtc_ws: the split-summary scratch (gtc_bytes), or nullptr where the grouped path does
+// not apply.
+static cudaError_t run_select(const hils::SelectArgs& a, void* gtc_ws, cudaStream_t st) {
   if (hils::select_tc_supported(a.d, a.h / a.g, a.top_k, a.bf16)) {
     hils::SelectArgs t = a;
     t.poll = g_wait_limit.load();
     return hils::run_select_tc(t, st);
+  }
+  if (gtc_ws) {
+    hils::GtcArgs g{};
+    g.q = static_cast<const __nv_bfloat16*>(a.q);
+    g.kbar = a.kbar; g.hbias = a.hbias; g.idx = a.idx; g.score = a.score; g.err = a.err;
+    const size_t half = align_up(hils::gtc_split_bytes(a.b, a.h, a.n_chunks, a.d));
+    g.kbar_hi = static_cast<__nv_bfloat16*>(gtc_ws);
+    g.kbar_lo = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(gtc_ws) + half);
+    g.b = a.b; g.h = a.h; g.g = a.g; g.n = a.n; g.d = a.d; g.n_chunks = a.n_chunks; g.top_k = a.top_k;
+    g.n_local = a.n_local; g.scale = a.scale; g.poll = g_wait_limit.load();
+    return hils::run_select_gtc(g, st);
   }
   return hils::run_select_simt(a, st);
 }
@@ -278,14 +306,15 @@ hils_status hils_select(const hils_shape* s, const void* q, const float* kbar, c
   const int C = s->seq_len / s->chunk;
   if (!q || !topk_idx || (C > 0 && (!kbar || !hbias))) return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || (C > 0 && !aligned16(kbar))) return HILS_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < kHeader || !aligned16(ws)) return HILS_ERR_WORKSPACE;
+  const size_t gb = gtc_bytes(s);
+  if (!ws || ws_bytes < kHeader + gb || !aligned16(ws)) return HILS_ERR_WORKSPACE;
   hils::SelectArgs a{};
   a.q = q; a.kbar = kbar; a.hbias = hbias; a.idx = topk_idx; a.score = topk_score;
   a.err = static_cast<unsigned*>(ws);
   a.b = s->batch; a.h = s->heads_q; a.g = s->heads_kv; a.n = s->seq_len; a.d = s->head_dim;
   a.n_chunks = C; a.top_k = s->top_k; a.scale = eff_scale(s); a.bf16 = s->dtype == HILS_BF16;
   a.n_local = n_local(s);
-  return cuda_status(run_select(a, (cudaStream_t)stream));
+  return cuda_status(run_select(a, gb ? static_cast<char*>(ws) + kHeader : nullptr, (cudaStream_t)stream));
 }
 
 hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const void* v,
@@ -323,7 +352,7 @@ hils_status hils_attend(const hils_shape* s, const void* q, const void* k, const
     se.b = s->batch; se.h = s->heads_q; se.g = s->heads_kv; se.n = s->seq_len; se.d = s->head_dim;
     se.n_chunks = C; se.top_k = s->top_k; se.scale = scale; se.bf16 = bf16; se.n_local = n_local(s);
     se.err = reinterpret_cast<unsigned*>(w);
-    if (run_select(se, cs) != cudaSuccess) return HILS_ERR_CUDA;
+    if (run_select(se, L.gtc != L.cm ? w + L.gtc : nullptr, cs) != cudaSuccess) return HILS_ERR_CUDA;
   }
   return cuda_status(run_prefill_attention(s, q, k, v, idx, ssel, out, lse_out, reinterpret_cast<unsigned*>(w),
                                            L.cm != L.total ? w + L.cm : nullptr, cs));

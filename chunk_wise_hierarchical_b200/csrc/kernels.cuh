@@ -37,6 +37,27 @@ struct SelectArgs {
   uint32_t poll;          // polls of a bounded wait before it gives up (tensor-core kernel)
 };
 cudaError_t run_select_simt(const SelectArgs& a, cudaStream_t st);
+// Tensor-core scores + group Top-K for G = 2, 4, 8 query heads per KV head (bf16, K <= 32):
+// the summaries are split into bf16 hi + lo copies (kbar_hi / kbar_lo, workspace) first.
+struct alignas(64) GtcArgs {
+  CUtensorMap tmap_q;          // Q as [b*h][N][d], 64 x 128 boxes (set by the launcher)
+  CUtensorMap tmap_hi;         // kbar_hi as [b*h][C][d], 64 x 64 boxes
+  CUtensorMap tmap_lo;
+  const __nv_bfloat16* q;      // [b,h,N,d]
+  const float* kbar;           // [b,h,C,d]
+  __nv_bfloat16* kbar_hi;      // [b,h,C,d] workspace
+  __nv_bfloat16* kbar_lo;
+  const float* hbias;          // [b,h,C]
+  int32_t* idx;                // [b,g,N,K]
+  float* score;                // [b,h,N,K] or nullptr
+  unsigned* err;
+  int b, h, g, n, d, n_chunks, top_k, n_local;
+  float scale;
+  uint32_t poll;
+};
+bool select_gtc_supported(int d, int G, int K, bool bf16);
+size_t gtc_split_bytes(int b, int h, int n_chunks, int d);  // bytes of one of kbar_hi / kbar_lo
+cudaError_t run_select_gtc(GtcArgs a, cudaStream_t st);
 // Tensor-core scores + Top-K (bf16, one query head per KV head).
 bool select_tc_supported(int d, int G, int K, bool bf16);
 cudaError_t run_select_tc(const SelectArgs& a, cudaStream_t st);

@@ -128,6 +128,36 @@ def test_select_one_head_per_group_bf16(kw):
 
 
 @pytest.mark.parametrize("kw", [
+    dict(batch=1, heads_q=8, heads_kv=2, seq_len=64 * 70 + 13, head_dim=128, top_k=32, qkv_std=0.5, needles=4),
+    dict(batch=2, heads_q=4, heads_kv=2, seq_len=64 * 66 + 40, head_dim=64, top_k=16),
+    dict(batch=1, heads_q=16, heads_kv=2, seq_len=64 * 80, head_dim=64, top_k=16, needles=4),
+    dict(batch=1, heads_q=8, heads_kv=1, seq_len=64 * 65 + 1, head_dim=128, top_k=7),
+])
+def test_select_grouped_heads_bf16(kw):
+    """bf16 with G = 2, 4, 8 scores every head on the tensor cores (split-bf16 summaries)
+    and keeps the group's Top-K by the max over heads: indices as the oracle's up to
+    near-ties, each head's scores of the selected chunks within 1e-4."""
+    inp = prefill_inputs(dtype="bf16", seed=23, **kw)
+    K, g = kw["top_k"], kw["heads_kv"]
+    G = kw["heads_q"] // g
+    kbar, hb = hils.summarize(inp.k.cuda(), inp.landmark.cuda())
+    rk, rh = O.summarize(inp.k, inp.landmark, 64)
+    idx, sc = hils.select(inp.q.cuda(), kbar, hb, K, g)
+    shat = O.chunk_scores(inp.q, rk, rh, 64)
+    _, key = O.select_topk(shat, g, K)
+    gi = idx.cpu().numpy()
+    check_indices(gi, key, K)
+    gsc = sc.cpu().numpy()
+    b_, h_, n_, _ = gsc.shape
+    bi, hi, ii, si = np.nonzero(np.repeat(gi, G, axis=1) >= 0)
+    chosen = gi[bi, hi // G, ii, si]
+    assert np.abs(gsc[bi, hi, ii, si] - shat[bi, hi, ii, chosen]).max() < 1e-4
+    assert np.all(gsc[np.repeat(gi, G, axis=1) < 0] == -np.inf)
+    n_eff = np.minimum(np.arange(n_) // 64, K)
+    assert np.array_equal((gi >= 0).sum(-1), np.broadcast_to(n_eff, gi.shape[:3]))
+
+
+@pytest.mark.parametrize("kw", [
     dict(batch=1, heads_q=2, heads_kv=2, seq_len=64 * 16 + 37, head_dim=64, top_k=8),
     dict(batch=1, heads_q=8, heads_kv=2, seq_len=64 * 12, head_dim=128, top_k=4, qkv_std=0.5),
 ])
