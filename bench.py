@@ -58,21 +58,25 @@ def decode_bytes(cfg, summary_bytes=4):
     return float(kv + summ + qo), float(kv)
 
 
-# DRAM bytes (read + write) per launch of the prefill attention kernel at the bench size,
-# from one ncu capture (`ncu --set full --clock-control none -k regex:attend_tc_kernel -s 3
-# -c 1 python bench.py --steps 3 --warmup 3 --no-decode --no-cpu`, summarised under
-# profiles/).  Reported only while the kernel's sources are the ones it was taken on.
+# DRAM bytes (read + write) per launch of the prefill attention kernel at the bench size
+# (attend_tc3_kernel for the 345M shape), from one ncu capture summarised under profiles/
+# (attend_tc3_kernel_prefill_345m.md).  Reported only while the kernel's sources are the
+# ones it was taken on.
 ATTEND_TRAFFIC = {
-    "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc.cu":
-                "7d38efcfbbc3491a04b890039c80d3d548f03906078c602df6d85e34c43e963a",
+    "sources": {"chunk_wise_hierarchical_b200/csrc/attend_tc3.cu":
+                "c7a1d131b1c13ee793f69feff2448454ba899db1bba06b02660749024742bc2b",
                 "chunk_wise_hierarchical_b200/csrc/tc_util.cuh":
-                "2c8199fc4ff66b314758faa3af3800696b99b5856f4f2dcdf03a90bd6e6727b6"},
-    "bytes": 276958976 + 57682688,
+                "ef2b1f54b29d8d04a25e377aec7307ed799b53c87ff99ab707d9d0d845134640",
+                "chunk_wise_hierarchical_b200/csrc/common.cuh":
+                "f19fe418aeaa91592e04d1c59c503e5fa51570749ec0ad3378b36b7762f2c5b4"},
+    "bytes": 275178496 + 52989440,
 }
 
 
 def attend_traffic():
     import hashlib
+    if ATTEND_TRAFFIC["bytes"] is None:
+        return None
     for rel, digest in ATTEND_TRAFFIC["sources"].items():
         with open(os.path.join(ROOT, rel), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest() != digest:
@@ -449,11 +453,14 @@ def needle_recall(needles, idx, group):
     return {"hits": int(hit.sum()), "needles": len(needles), "fraction": round(float(hit.float().mean()), 4)}
 
 
-def run_prefill_gqa(dev, steps=5, warmup=3):
+def run_prefill_gqa(dev, steps=5, warmup=3, seq_len=None):
     """The 7B-shaped GQA prefill (b1 h32 g8 N32768 d128 K32): per-stage device times and
-    TFLOP/s of the same algorithmic FLOP count, reported beside the headline step."""
+    TFLOP/s of the same algorithmic FLOP count, reported beside the headline step.
+    seq_len shortens the sequence (a reduced case for profiling, not a bench line)."""
     import chunk_wise_hierarchical_b200 as hils
-    cfg = CONFIGS["prefill_7b_gqa"]
+    cfg = dict(CONFIGS["prefill_7b_gqa"])
+    if seq_len:
+        cfg["seq_len"] = seq_len
     inp = prefill_inputs(seed=0, device=dev, **cfg)
     q, k, v, lm = inp.q, inp.k, inp.v, inp.landmark
     b, h, n, d = q.shape
@@ -476,7 +483,7 @@ def run_prefill_gqa(dev, steps=5, warmup=3):
             times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(3)])
     med = [statistics.median(t[i] for t in times) for i in range(3)]
     flops = algorithmic_flops(b, h, n, d, K)
-    return {"workload": "prefill_7b_gqa: batch 1, 32 query heads / 8 KV heads, N 32768, d 128, top-k 32, bf16",
+    return {"workload": f"prefill_7b_gqa: batch 1, 32 query heads / 8 KV heads, N {n}, d 128, top-k 32, bf16",
             "ms_per_step": round(sum(med), 4), "needle_recall": needle_recall(inp.needles, idx, h // g),
             "stage_ms": {"summarize": round(med[0], 4), "select": round(med[1], 4), "attend_selected": round(med[2], 4)},
             "tflops": round(flops / (sum(med) * 1e-3) / 1e12, 3),
@@ -484,13 +491,15 @@ def run_prefill_gqa(dev, steps=5, warmup=3):
             "timing": "CUDA events per stage, median of %d steps, L2 flushed between steps" % steps}
 
 
-def run_training(dev, steps=5, warmup=3):
+def run_training(dev, steps=5, warmup=3, seq_len=None):
     """The training workload (b2 h16 N16384 d128 K16, bf16): one forward (summaries,
     selection, attention with log Zhat) and one hils_backward per step, with dO ~ N(0,1).
     Backward algorithmic FLOPs = 2.5 x the forward's: per (query, key) pair the forward
     does 4d (QK^T, PV) and the backward 10d (QK^T and dO V^T recomputed, dV, dK, dQ)."""
     import chunk_wise_hierarchical_b200 as hils
-    cfg = CONFIGS["train_16k"]
+    cfg = dict(CONFIGS["train_16k"])
+    if seq_len:
+        cfg["seq_len"] = seq_len
     inp = prefill_inputs(seed=0, device=dev, **cfg)
     q, k, v, lm = inp.q, inp.k, inp.v, inp.landmark
     b, h, n, d = q.shape
@@ -520,7 +529,7 @@ def run_training(dev, steps=5, warmup=3):
     fwd = statistics.median(t[0] for t in times)
     bwd = statistics.median(t[1] for t in times)
     flops = algorithmic_flops(b, h, n, d, K)
-    return {"workload": "train_16k: batch 2, 16 heads, N 16384, d 128, top-k 16, bf16 N(0,1), dO N(0,1)",
+    return {"workload": f"train_16k: batch 2, 16 heads, N {n}, d 128, top-k 16, bf16 N(0,1), dO N(0,1)",
             "forward_ms": round(fwd, 3), "backward_ms": round(bwd, 3),
             "forward_tflops": round(flops / (fwd * 1e-3) / 1e12, 2),
             "backward_tflops": round(2.5 * flops / (bwd * 1e-3) / 1e12, 2),
@@ -604,8 +613,8 @@ def run_ours(args):
                                              "frac_hbm": round(r["gbs"] / hbm, 4)} for k, r in dec.items()}}))
         return
     pre = run_prefill(args, ws_world, rank, local)
-    gqa = run_prefill_gqa(torch.device("cuda", local)) if not args.no_gqa else None
-    train = run_training(torch.device("cuda", local)) if not args.no_train else None
+    gqa = run_prefill_gqa(torch.device("cuda", local), seq_len=args.gqa_seq) if not args.no_gqa else None
+    train = run_training(torch.device("cuda", local), seq_len=args.train_seq) if not args.no_train else None
     cpu = cpu1 = otimes = None
     if rank == 0 and ws_world == 1 and not args.no_cpu:
         cpu = cpu_baseline(args.cpu_seconds)                 # every host core
@@ -716,6 +725,10 @@ def main():
     ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the 7B-shaped GQA prefill line")
+    ap.add_argument("--gqa-seq", type=int, default=None,
+                    help="shorter sequence for the GQA line (a reduced case for profiling)")
+    ap.add_argument("--train-seq", type=int, default=None,
+                    help="shorter sequence for the training line (a reduced case for profiling)")
     ap.add_argument("--no-train", action="store_true", help="skip the forward + backward training line")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
