@@ -602,8 +602,10 @@ def run_ours(args):
     dec = {}
     if not args.no_decode:
         for name in args.decode_configs.split(","):
-            # three rotating caches (each larger than L2 from 128K up) keep every step's reads in HBM
-            r = run_decode(name, 3, torch.device("cuda", local))
+            # three rotating caches (each larger than L2 from 128K up) keep every step's reads in
+            # HBM; from 1M tokens on, one cache (about 34 GB) is far beyond L2 by itself
+            big = CONFIGS[name]["batch"] * CONFIGS[name]["seq_len"] > (1 << 22)
+            r = run_decode(name, 1 if big else 3, torch.device("cuda", local))
             dec[name] = r[torch.float32]
             dec[name + "_bf16_summaries"] = r[torch.bfloat16]
     if args.decode_only:
@@ -722,7 +724,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode configurations")
-    ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k")
+    ap.add_argument("--decode-configs", default="decode_32k,decode_128k,decode_512k,decode_1m,decode_4m")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the 7B-shaped GQA prefill line")
     ap.add_argument("--gqa-seq", type=int, default=None,

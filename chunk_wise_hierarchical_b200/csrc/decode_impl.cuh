@@ -29,7 +29,6 @@ constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kMaxRange = 256;          // candidate chunks per scan CTA, at most ...
 constexpr int kMinRange = 16;           // ... and at least
 constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B200
-constexpr int kMergeN = 256;            // keys one warp sorts at once in the fallback merge
 
 
 constexpr int kMaxListsPerLane = 4;
@@ -265,80 +264,72 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       }
     }
   };
-  if (a.nsplit <= 32 * kMaxListsPerLane) {
-    // tournament: the lists are sorted, so each step is a warp max over the lists' heads
-    // (keys are unique: they carry the chunk index).  Lane l follows lists l, l + 32, ...
-    // straight from global memory, holding each list's head and the key after it, and
-    // fetching the next one as soon as a head is taken.
-    for (int gi = warp; gi < a.g; gi += kScanWarps) {
-      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
-      int pos[kMaxListsPerLane];
-      unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
+  // Tournament over n_lists sorted lists of K keys (list l at parts + l K): each step is a
+  // warp max over the lists' heads (keys are unique: they carry the chunk index).  Lane l
+  // follows lists l, l + 32, ... straight from global memory, holding each list's head and
+  // the key after it, and fetching the next one as soon as a head is taken.  Returns the
+  // best K in descending order: slot lane in r0, slot lane + 32 in r1 (0: empty).
+  auto tournament = [&](const unsigned long long* parts, int n_lists, unsigned long long& r0,
+                        unsigned long long& r1) {
+    int pos[kMaxListsPerLane];
+    unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
+#pragma unroll
+    for (int m = 0; m < kMaxListsPerLane; ++m) {
+      const int l = lane + 32 * m;
+      const bool live = l < n_lists;
+      pos[m] = 0;
+      head[m] = live ? __ldcg(parts + (size_t)l * K) : 0ull;
+      next[m] = live && K > 1 ? __ldcg(parts + (size_t)l * K + 1) : 0ull;
+    }
+    r0 = 0ull;
+    r1 = 0ull;
+    for (int s = 0; s < K; ++s) {
+      unsigned long long lb = head[0];
+#pragma unroll
+      for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
+      unsigned long long wb = lb;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long y = shfl_xor_u64(wb, o);
+        wb = y > wb ? y : wb;
+      }
+      if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
 #pragma unroll
       for (int m = 0; m < kMaxListsPerLane; ++m) {
-        const int l = lane + 32 * m;
-        const bool live = l < a.nsplit;
-        pos[m] = 0;
-        head[m] = live ? __ldcg(parts + (size_t)l * K) : 0ull;
-        next[m] = live && K > 1 ? __ldcg(parts + (size_t)l * K + 1) : 0ull;
-      }
-      unsigned long long res0 = 0ull, res1 = 0ull;
-      for (int s = 0; s < K; ++s) {
-        unsigned long long lb = head[0];
-#pragma unroll
-        for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
-        unsigned long long wb = lb;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const unsigned long long y = shfl_xor_u64(wb, o);
-          wb = y > wb ? y : wb;
-        }
-        if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
-#pragma unroll
-        for (int m = 0; m < kMaxListsPerLane; ++m) {
-          if (head[m] == wb) {  // this lane's list m holds the winner: advance it
-            ++pos[m];
-            head[m] = next[m];
-            next[m] = pos[m] + 1 < K ? __ldcg(parts + (size_t)(lane + 32 * m) * K + pos[m] + 1) : 0ull;
-          }
-        }
-        if ((s & 31) == lane) {
-          if (s < 32) res0 = wb;
-          else res1 = wb;
+        if (head[m] == wb) {  // this lane's list m holds the winner: advance it
+          ++pos[m];
+          head[m] = next[m];
+          next[m] = pos[m] + 1 < K ? __ldcg(parts + (size_t)(lane + 32 * m) * K + pos[m] + 1) : 0ull;
         }
       }
-      emit(gi, res0, res1);
+      if ((s & 31) == lane) {
+        if (s < 32) r0 = wb;
+        else r1 = wb;
+      }
     }
-  } else {
-    // running best K + the next slice of keys, sorted by the warp
-    for (int gi = warp; gi < a.g; gi += kScanWarps) {
-      const unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
-      constexpr int ME = kMergeN / 32;
-      unsigned long long v[ME];
-#pragma unroll
-      for (int e = 0; e < ME; ++e) v[e] = 0ull;
-      for (int start = 0; start < n_all; start += kMergeN - K) {
-        const int take = min(kMergeN - K, n_all - start);
-#pragma unroll
-        for (int e = 0; e < ME; ++e) {
-          const int i = lane * ME + e;
-          if (i >= K) v[e] = i - K < take ? __ldcg(parts + start + i - K) : 0ull;
-        }
-        warp_sort_desc<ME>(v);
+  };
+  constexpr int kTour = 32 * kMaxListsPerLane;  // lists one tournament takes
+  for (int gi = warp; gi < a.g; gi += kScanWarps) {
+    unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
+    unsigned long long r0, r1;
+    if (a.nsplit <= kTour) {
+      tournament(parts, a.nsplit, r0, r1);
+    } else {
+      // more ranges than one tournament takes: each group of kTour lists gives its best K,
+      // written back as list g (a slot of group 0, already consumed), then a final tournament
+      // over the groups' lists
+      const int n_groups = (a.nsplit + kTour - 1) / kTour;
+      for (int grp = 0; grp < n_groups; ++grp) {
+        tournament(parts + (size_t)grp * kTour * K, min(kTour, a.nsplit - grp * kTour), r0, r1);
+        __syncwarp();
+        if (lane < K) __stcg(parts + (size_t)grp * K + lane, r0);
+        if (lane + 32 < K) __stcg(parts + (size_t)grp * K + lane + 32, r1);
+        __threadfence_block();
+        __syncwarp();
       }
-      // slot s sits in lane s / ME, register s % ME: move slots lane and lane + 32 here
-      unsigned long long k0 = 0ull, k1 = 0ull;
-#pragma unroll
-      for (int e = 0; e < ME; ++e) {
-        const unsigned long long x0 = __shfl_sync(0xffffffffu, (uint32_t)v[e], lane / ME) |
-                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), lane / ME) << 32);
-        const unsigned long long x1 = __shfl_sync(0xffffffffu, (uint32_t)v[e], (lane + 32) / ME) |
-                                      ((unsigned long long)__shfl_sync(0xffffffffu, (uint32_t)(v[e] >> 32), (lane + 32) / ME) << 32);
-        if (lane % ME == e) k0 = x0;
-        if ((lane + 32) % ME == e) k1 = x1;
-      }
-      emit(gi, k0, k1);
+      tournament(parts, n_groups, r0, r1);
     }
+    emit(gi, r0, r1);
   }
   if constexpr (G > 1) {
     __syncthreads();  // the selection written above is read back below

@@ -44,6 +44,11 @@ CONFIGS = {
                         chunk=64, top_k=16, dtype="bf16"),
     "decode_512k": dict(batch=8, heads_q=16, heads_kv=16, seq_len=524288, head_dim=64,
                         chunk=64, top_k=16, dtype="bf16"),
+    # the longer contexts the pages extrapolate decode to: about 34 GB of K/V pages each
+    "decode_1m": dict(batch=8, heads_q=16, heads_kv=16, seq_len=1048576, head_dim=64,
+                      chunk=64, top_k=16, dtype="bf16"),
+    "decode_4m": dict(batch=2, heads_q=16, heads_kv=16, seq_len=4194304, head_dim=64,
+                      chunk=64, top_k=16, dtype="bf16"),
 }
 
 _DT = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -353,6 +353,18 @@ def test_decode_512k_full_size_sampled():
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name,pair", [("decode_1m", (5, 9)), ("decode_4m", (1, 4))])
+def test_decode_1m_4m_full_size_sampled(name, pair):
+    """The longer contexts (1M tokens x 8 sequences, 4M tokens x 2): the scan runs 74 and
+    296 ranges per sequence, the latter through the sorted-slice merge."""
+    cfg = CONFIGS[name]
+    di = decode_inputs(device="cuda", seed=0, **cfg)
+    out, idx = _gpu_decode(di, cfg["top_k"])
+    _check_decode(di, out, idx, cfg["top_k"], [pair])
+    del di, out, idx
+    torch.cuda.empty_cache()
+
+
 def test_decode_equals_prefill_row_on_gpu():
     """P10 on the GPU: a decode step at position t reproduces prefill row t."""
     inp = prefill_inputs(1, 4, 2, 640, 64, top_k=4, dtype="bf16", seed=12, needles=2)
