@@ -1,8 +1,9 @@
 """The give-up path of the bounded device waits, on the GPU.
 
 With the wait limit at 0 every ordinary mbarrier wait of the tensor-core
-kernels (select with one query head per KV head, prefill attention for head
-dim 64 and 128) gives up at its first poll.  The kernel then records
+kernels gives up at its first poll: select with one query head per KV head
+and with G = 4 grouped heads, prefill attention for head dim 64 (the
+row-owner kernel) and 128 (the chunk-major kernel).  The kernel then records
 HILS_ERR_DEVICE_TIMEOUT in the workspace's error word, waits for the copies
 and MMAs it already issued, releases its tensor memory and returns.  The test
 checks that status and that the next calls on the same context, with the
@@ -24,9 +25,9 @@ pytestmark = pytest.mark.gpu
 HILS_OK, HILS_ERR_DEVICE_TIMEOUT = 0, 6
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_forced_give_up_then_a_normal_call(d):
-    b, h, g, n, K = 1, 2, 2, 64 * 6 + 10, 2
+@pytest.mark.parametrize("d,h,g,n", [(64, 2, 2, 64 * 6 + 10), (128, 2, 2, 64 * 6 + 10), (128, 8, 2, 64 * 65 + 3)])
+def test_forced_give_up_then_a_normal_call(d, h, g, n):
+    b, K = 1, 2
     inp = prefill_inputs(batch=b, heads_q=h, heads_kv=g, seq_len=n, head_dim=d, top_k=K, dtype="bf16", seed=5)
     q, k, v, lm = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.landmark))
     sh = make_shape(b, h, g, d, n, K, HILS_BF16)
