@@ -664,10 +664,7 @@ __global__ void __launch_bounds__(256) cm_fuse_kernel(const __grid_constant__ Cm
   float Z = 0.f, acc[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-  auto add = [&](long long pr, float x) {
-    const float w = expf(x - M);
-    Z += w;
-    const uint4 pv = __ldg(reinterpret_cast<const uint4*>(a.part + pr * D + ln * 8));
+  auto accumulate = [&](float w, const uint4& pv) {
     const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -679,11 +676,33 @@ __global__ void __launch_bounds__(256) cm_fuse_kernel(const __grid_constant__ Cm
   for (int l = 0; l < a.n_local && own - l >= 0; ++l) {
     const int c = own - l;
     const long long pr = ((long long)(bg * a.c_all + c) * a.tl) * 128 + (long long)(i - c * kChunk) * G + hh;
-    add(pr, __ldg(a.plse + pr));
+    const float w = expf(__ldg(a.plse + pr) - M);
+    Z += w;
+    accumulate(w, __ldg(reinterpret_cast<const uint4*>(a.part + pr * D + ln * 8)));
   }
-  for (int s = 0; s < K; ++s) {
-    const int p = __ldg(pos + s);
-    if (p >= 0) add((long long)p + hh, __ldg(sc + s));
+  // the selections in batches of 8: their positions and scores, then their 8 partial rows,
+  // all in flight before any is used
+  for (int s0 = 0; s0 < K; s0 += 8) {
+    int p[8];
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      p[u] = s0 + u < K ? __ldg(pos + s0 + u) : -1;
+      x[u] = p[u] >= 0 ? __ldg(sc + s0 + u) : 0.f;
+    }
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = p[u] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.part + ((long long)p[u] + hh) * D + ln * 8))
+                       : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (p[u] >= 0) {
+        const float w = expf(x[u] - M);
+        Z += w;
+        accumulate(w, v[u]);
+      }
+    }
   }
   const float inv = 1.0f / Z;
   uint4 o;

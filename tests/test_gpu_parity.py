@@ -224,6 +224,7 @@ def test_prefill_7b_gqa_full_size_sampled():
     dict(batch=1, heads_q=4, heads_kv=1, seq_len=64 * 14, head_dim=128, top_k=3, dtype="f32", window=192),
     dict(batch=2, heads_q=8, heads_kv=2, seq_len=64 * 12 + 40, head_dim=64, top_k=8, dtype="bf16", window=512),
     dict(batch=1, heads_q=2, heads_kv=2, seq_len=300, head_dim=64, top_k=2, dtype="f32", window=64),
+    dict(batch=1, heads_q=8, heads_kv=2, seq_len=64 * 18 + 5, head_dim=128, top_k=4, dtype="bf16", window=192),
 ])
 def test_prefill_sliding_window_local_branch(kw):
     """The chunk-aligned sliding-window local branch (notes sections 5.2-5.3)."""
