@@ -5,7 +5,7 @@
 // c < floor(i / B) + 1 - n_local, ties to the lower chunk index.)
 //
 // One CTA takes 128 queries of one (sequence, KV head).  The summaries are split
-// once into bf16 hi + lo parts (cm_split_kernel), so every head's score tile is
+// once into bf16 hi + lo parts (gtc_split_kernel), so every head's score tile is
 // S_h = Q_h hi_h^T + Q_h lo_h^T on the tensor cores, accumulated in fp32 in its
 // own tensor-memory region (G regions of kNc = 64 chunk columns).  Q_h, hi_h and
 // lo_h come by TMA into a two-deep ring of stages, one (tile, head) pair per stage.

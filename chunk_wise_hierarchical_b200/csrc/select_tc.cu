@@ -158,17 +158,35 @@ __global__ void __launch_bounds__(kSelThreads) select_tc_kernel(SelectArgs a) {
     }
     phase ^= 1u;
     tc::fence_after_sync();
-    // this tile's candidates, 32 TMEM columns at a time
+    // this tile's candidates, 32 TMEM columns at a time.  The candidates above the list's
+    // last score are first queued, in chunk order, in shared memory (the summary tiles are
+    // free once the MMA has read them); the queue is then inserted in order, each entry
+    // checked again against the rising threshold, so every decision is the one a candidate-
+    // by-candidate insertion would take.  A warp then runs as many insertions as its longest
+    // queue rather than one for every candidate some lane keeps.
+    float* qx = reinterpret_cast<float*>(sm + (sHi - sQ));  // [32][128], thread-minor
+    int* qc = reinterpret_cast<int*>(qx + 32 * kSelThreads);
 #pragma unroll 1
     for (int cb = 0; cb < nc; cb += 32) {
       float sv[32];
       tc::tmem_ld32(tmem + cb + lane_off, sv);
       tc::tmem_wait_ld();
+      const float thr = S[KP - 1];
+      int cnt = 0;
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         const int c = c0 + cb + u;
         const float x = fmaf(sv[u], a.scale, s_h[cb + u]);
-        if (c < n_cand && x > S[KP - 1]) sorted_insert_f(S, I, x, c);
+        if (c < n_cand && x > thr) {
+          qx[cnt * kSelThreads + t] = x;
+          qc[cnt * kSelThreads + t] = c;
+          ++cnt;
+        }
+      }
+#pragma unroll 1
+      for (int e = 0; e < cnt; ++e) {
+        const float x = qx[e * kSelThreads + t];
+        if (x > S[KP - 1]) sorted_insert_f(S, I, x, qc[e * kSelThreads + t]);
       }
     }
     tc::fence_before_sync();
