@@ -26,16 +26,19 @@
 // queries they come from, and a tile's result leaves the SM without a read-modify-
 // write of an accumulator, so tiles are independent of each other.
 //
-// attend_cm_kernel: one persistent CTA per SM walks tiles t = blockIdx.x + k gridDim.x.
-// Warp roles (512 threads), synchronised by mbarriers with bounded waits:
-//   warp 0 lane 0   TMA producer: K_c and V_c into a stage of their own, on a change of chunk
+// attend_cm_kernel: one persistent CTA per SM.  The tile list is cut into blocks of U
+// consecutive tiles, block k going to CTA k % gridDim.x, so a CTA's consecutive items
+// mostly share their chunk.  Warp roles (512 threads), synchronised by mbarriers with
+// bounded waits:
+//   warp 0 lane 0   TMA producer: K_c and V_c into a K/V stage (which also holds a tile of
+//                   ones), once per change of chunk; a stage is refilled after the last
+//                   P.V that read it has completed
 //   warp 1 lane 0   MMA issuer: S(0), S(1), then P.V(j), S(j + 2), ...
-//   warps 2-3       gather of the tile's Q rows into the stage (cp.async, fenced for
-//                   the async proxy, signalled one item late so two stay in flight)
+//   warps 2-3       gather of the tile's Q rows into a Q stage (whole-row cp.async, each
+//                   copy arriving on the stage's barrier when it lands); a Q stage is
+//                   released by the softmax once S has been read
 //   warps 4-11      two softmax warpgroups on alternate items
 //   warps 12-15     epilogue: tensor memory -> registers -> bf16 partial rows in global
-// A stage holds Q rows, K_c, V_c and a tile of ones; it is refilled once P.V of its
-// item has completed.
 #include <cudaTypedefs.h>
 
 #include <mutex>

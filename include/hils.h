@@ -174,11 +174,16 @@ HILS_API hils_status hils_summarize_paged(const hils_shape* shape, const void* k
  *   topk_score  [batch, heads_q, seq_len, top_k] fp32 or NULL: each head's
  *               own shat of the selected chunks (-inf in unused slots)
  *   ws          workspace of hils_workspace_size(HILS_OP_SELECT) bytes,
- *               zero-filled before first use: it holds only the sticky
- *               error word read by hils_device_status
- * kbar must be 16-byte aligned.  For bf16 with heads_q == heads_kv the
- * scores run on the tensor cores with the fp32 summaries split into two
- * bf16 parts (score error near 2^-17 |q||kbar|).
+ *               zero-filled before first use: it holds the sticky error
+ *               word read by hils_device_status and, for the grouped
+ *               tensor-core path below, the bf16 hi and lo parts of the
+ *               summaries (rewritten by every call)
+ * kbar must be 16-byte aligned.  For bf16 the scores run on the tensor
+ * cores with the fp32 summaries split into two bf16 parts (score error
+ * near 2^-17 |q||kbar|) when heads_q == heads_kv, and when heads_q /
+ * heads_kv is 2, 4 or 8 with top_k <= 16 (up to 32 where the candidate
+ * records fit in shared memory), C >= 64 and seq_len >= 128;
+ * other shapes score on the CUDA cores in fp32.
  */
 HILS_API hils_status hils_select(const hils_shape* shape, const void* q, const float* kbar,
                         const float* hbias, int32_t* topk_idx, float* topk_score, void* ws,
@@ -199,7 +204,11 @@ HILS_API hils_status hils_select(const hils_shape* shape, const void* q, const f
  *                chunks' shat and the local branch's exact log-mass), the
  *                row statistic a backward pass needs
  *   topk_idx_out [batch, heads_kv, seq_len, top_k] int32 or NULL
- *   ws           workspace of hils_workspace_size(HILS_OP_ATTEND) bytes
+ *   ws           workspace of hils_workspace_size(HILS_OP_ATTEND) bytes,
+ *                zero-filled before first use: the error word, the
+ *                summaries, the selection and its scores, the select
+ *                scratch of hils_select and the chunk-major scratch of
+ *                hils_attend_selected (all rewritten by every call)
  */
 HILS_API hils_status hils_attend(const hils_shape* shape, const void* q, const void* k, const void* v,
                         const void* landmark_q, void* out, float* lse_out, int32_t* topk_idx_out,
@@ -222,6 +231,12 @@ HILS_API hils_status hils_attend(const hils_shape* shape, const void* q, const v
  *   lse_out      [batch, heads_q, seq_len] fp32 or NULL: log Zhat_i as in
  *                hils_attend
  *   ws           workspace of hils_workspace_size(HILS_OP_ATTEND_SELECTED)
+ *                bytes, zero-filled before first use: the error word and,
+ *                for bf16 shapes that take the chunk-major path (the
+ *                selections bucketed by chunk into 128-row tiles, a bf16
+ *                partial output per selection, fused per row afterwards),
+ *                its bucket counts, tile list, selection positions and
+ *                partials; other shapes use the error word only
  */
 HILS_API hils_status hils_attend_selected(const hils_shape* shape, const void* q, const void* k,
                                           const void* v, const int32_t* topk_idx,
