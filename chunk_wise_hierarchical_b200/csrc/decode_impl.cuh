@@ -19,6 +19,8 @@
 // Tickets are reset by the CTA that consumes them, so both kernels can be
 // replayed (CUDA graphs) without clearing the workspace.
 #pragma once
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -32,6 +34,7 @@ constexpr int kScanCtasTarget = 4 * 148;  // about four scan CTAs per SM of a B2
 
 
 constexpr int kMaxListsPerLane = 4;
+constexpr int kStageKeys = 512;         // keys of range lists staged in shared memory per merging warp
 constexpr int kMaxDecodeLocal = 16;     // local-branch chunks a decode step supports
 
 
@@ -78,9 +81,22 @@ __device__ __forceinline__ void warp_sort_desc(unsigned long long (&v)[E]) {
     }
   }
 }
+// The largest of the warp's 64-bit keys: two 32-bit warp reductions (redux.sync), the
+// high words first, then the low words among the lanes that hold the largest high word.
+__device__ __forceinline__ unsigned long long warp_max_key(unsigned long long v) {
+  const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32));
+  const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32) == hi ? (uint32_t)v : 0u);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
 // Top-K of one KV head over this CTA's range: the key of chunk j is the max over the
 // group's heads of s_score[j][head] (a NaN, from a bad page, makes the key 0).  Writes
 // the K best keys (0 where the range has fewer) in descending order.
+// E <= 2: a bitonic sort of the warp's 32 E keys.  E >= 4: each lane sorts its own E keys,
+// then each of the K steps takes the warp's largest head (keys are unique: they carry the
+// chunk index) and the lane that held it moves to its next key -- K steps of two warp
+// reductions instead of the sort's 15 exchange stages of 2 E shuffles each, which, with
+// every scan warp of the SM sorting at once, queue on the SM's shuffle unit.
 template <int E, int G>
 __device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, int nc, int c_lo, int K,
                                            unsigned long long* out) {
@@ -103,13 +119,37 @@ __device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, 
     }
     v[e] = key;
   }
-  warp_sort_desc<E>(v);
+  if constexpr (E <= 2) {
+    warp_sort_desc<E>(v);
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = lane * E + e;
-    if (i < K) out[i] = v[e];
+    for (int e = 0; e < E; ++e) {
+      const int i = lane * E + e;
+      if (i < K) out[i] = v[e];
+    }
+    for (int i = 32 * E + lane; i < K; i += 32) out[i] = 0ull;
+  } else {
+    // odd-even transposition sort of the lane's keys, descending
+#pragma unroll
+    for (int r = 0; r < E; ++r)
+#pragma unroll
+      for (int e = r & 1; e + 1 < E; e += 2) {
+        const unsigned long long x = v[e], y = v[e + 1];
+        v[e] = x > y ? x : y;
+        v[e + 1] = x > y ? y : x;
+      }
+    int s = 0;
+    for (; s < K; ++s) {
+      const unsigned long long wb = warp_max_key(v[0]);
+      if (wb == 0ull) break;  // every key taken (warp-uniform)
+      if (lane == 0) out[s] = wb;
+      if (v[0] == wb) {
+#pragma unroll
+        for (int e = 0; e + 1 < E; ++e) v[e] = v[e + 1];
+        v[E - 1] = 0ull;
+      }
+    }
+    for (int i = s + lane; i < K; i += 32) out[i] = 0ull;
   }
-  for (int i = 32 * E + lane; i < K; i += 32) out[i] = 0ull;
 }
 
 // Scan: CTA per (sequence, range of chunks), all heads.  A page's summaries of all
@@ -247,30 +287,45 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
   __threadfence();
 
   // ---- last CTA of the sequence: per KV head, merge the ranges' lists ----
+  // Every dependent round trip to L2 costs about as much here as the merge's arithmetic, so
+  // the merge is laid out to make few of them: the lists' leading keys are staged in shared
+  // memory with all loads in flight at once, a warp stages the lists of two heads together,
+  // and the block-table lookups of both heads' selections are issued together.
   const int lane = t & 31;
   const int n_all = a.nsplit * K;
-  // the selected keys of slots lane and lane + 32, in descending order (0: empty)
-  auto emit = [&](int gi, unsigned long long k0, unsigned long long k1) {
+  unsigned long long* win = reinterpret_cast<unsigned long long*>(s_score) + (size_t)warp * kStageKeys;
+  // Copies the first KW keys of each of n_lists lists of nh heads (head j's lists at
+  // parts[j] + l K) into the window: head j, list l, key p at win[(j n_lists + l) KW + p].
+  auto stage = [&](const unsigned long long* const (&parts)[2], int nh, int n_lists, int KW) {
+    const int n_win = n_lists * KW, n_tot = nh * n_win;
+    __syncwarp();  // the window's previous contents have been read
+    for (int x0 = 0; x0 < n_tot; x0 += 32 * 16) {
+      unsigned long long tmp[16];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int s = lane + 32 * r;
-      const unsigned long long key = r ? k1 : k0;
-      if (s < K) {
-        const int c = key ? (int)key_chunk(key) : -1;
-        a.idx[((size_t)bi * a.g + gi) * K + s] = c;
-        a.sel_page[((size_t)bi * a.g + gi) * K + s] = c >= 0 ? bt[c] : -1;
-        // G = 1: the selection key is the head's own score
-        if (G == 1) a.ssel[((size_t)bi * a.h + gi) * K + s] = key ? unorderable((uint32_t)(key >> 32)) : -INFINITY;
+      for (int u = 0; u < 16; ++u) {
+        const int x = x0 + 32 * u + lane;
+        const int j = x >= n_win, xx = x - j * n_win;
+        tmp[u] = x < n_tot ? __ldcg(parts[j] + (size_t)(xx / KW) * K + xx % KW) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int x = x0 + 32 * u + lane;
+        if (x < n_tot) win[x] = tmp[u];
       }
     }
+    __syncwarp();
   };
-  // Tournament over n_lists sorted lists of K keys (list l at parts + l K): each step is a
-  // warp max over the lists' heads (keys are unique: they carry the chunk index).  Lane l
-  // follows lists l, l + 32, ... straight from global memory, holding each list's head and
-  // the key after it, and fetching the next one as soon as a head is taken.  Returns the
-  // best K in descending order: slot lane in r0, slot lane + 32 in r1 (0: empty).
-  auto tournament = [&](const unsigned long long* parts, int n_lists, unsigned long long& r0,
-                        unsigned long long& r1) {
+  // Tournament over n_lists sorted lists of K keys (list l at parts + l K), whose first KW
+  // keys are staged at w + l KW: each step is a warp max over the lists' heads (keys are
+  // unique: they carry the chunk index), so a step waits on shared memory only; a list that
+  // wins more than KW - 1 times reads on from global memory.  Lane l follows lists l, l + 32,
+  // ..., holding each list's head and the key after it.  Returns the best K in descending
+  // order: slot lane in r0, slot lane + 32 in r1 (0: empty).
+  auto tournament = [&](const unsigned long long* parts, const unsigned long long* w, int n_lists, int KW,
+                        unsigned long long& r0, unsigned long long& r1) {
+    auto key_at = [&](int l, int p) -> unsigned long long {
+      return p < KW ? w[l * KW + p] : p < K ? __ldcg(parts + (size_t)l * K + p) : 0ull;
+    };
     int pos[kMaxListsPerLane];
     unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
 #pragma unroll
@@ -278,8 +333,8 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       const int l = lane + 32 * m;
       const bool live = l < n_lists;
       pos[m] = 0;
-      head[m] = live ? __ldcg(parts + (size_t)l * K) : 0ull;
-      next[m] = live && K > 1 ? __ldcg(parts + (size_t)l * K + 1) : 0ull;
+      head[m] = live ? key_at(l, 0) : 0ull;
+      next[m] = live ? key_at(l, 1) : 0ull;
     }
     r0 = 0ull;
     r1 = 0ull;
@@ -287,19 +342,14 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       unsigned long long lb = head[0];
 #pragma unroll
       for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
-      unsigned long long wb = lb;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long y = shfl_xor_u64(wb, o);
-        wb = y > wb ? y : wb;
-      }
+      const unsigned long long wb = warp_max_key(lb);
       if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
 #pragma unroll
       for (int m = 0; m < kMaxListsPerLane; ++m) {
         if (head[m] == wb) {  // this lane's list m holds the winner: advance it
           ++pos[m];
           head[m] = next[m];
-          next[m] = pos[m] + 1 < K ? __ldcg(parts + (size_t)(lane + 32 * m) * K + pos[m] + 1) : 0ull;
+          next[m] = key_at(lane + 32 * m, pos[m] + 1);
         }
       }
       if ((s & 31) == lane) {
@@ -308,28 +358,74 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       }
     }
   };
+  // Writes the selections of heads gi[0] and gi[1] (gi >= g: none): keys r[j][0] for slot
+  // lane and r[j][1] for slot lane + 32, in descending order (0: empty).  The four block-table
+  // reads are issued before any is used.
+  auto emit = [&](const int (&gi)[2], const unsigned long long (&r)[2][2]) {
+    int c[2][2], pg[2][2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const bool live = gi[j] < a.g && lane + 32 * q < K;
+        c[j][q] = live && r[j][q] ? (int)key_chunk(r[j][q]) : -1;
+        pg[j][q] = c[j][q] >= 0 ? bt[c[j][q]] : -1;
+      }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int sl = lane + 32 * q;
+        if (gi[j] >= a.g || sl >= K) continue;
+        a.idx[((size_t)bi * a.g + gi[j]) * K + sl] = c[j][q];
+        a.sel_page[((size_t)bi * a.g + gi[j]) * K + sl] = pg[j][q];
+        // G = 1: the selection key is the head's own score
+        if (G == 1)
+          a.ssel[((size_t)bi * a.h + gi[j]) * K + sl] = r[j][q] ? unorderable((uint32_t)(r[j][q] >> 32)) : -INFINITY;
+      }
+  };
   constexpr int kTour = 32 * kMaxListsPerLane;  // lists one tournament takes
-  for (int gi = warp; gi < a.g; gi += kScanWarps) {
-    unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + gi) * n_all;
-    unsigned long long r0, r1;
-    if (a.nsplit <= kTour) {
-      tournament(parts, a.nsplit, r0, r1);
-    } else {
-      // more ranges than one tournament takes: each group of kTour lists gives its best K,
-      // written back as list g (a slot of group 0, already consumed), then a final tournament
-      // over the groups' lists
+  if (a.nsplit <= kTour) {
+    // heads in pairs (warp, warp + kScanWarps), then (warp + 2 kScanWarps, ...), ...: each
+    // head's lists get half the window
+    const int KW = max(1, min(K, (kStageKeys / 2) / a.nsplit));
+    for (int g0 = warp; g0 < a.g; g0 += 2 * kScanWarps) {
+      const int gi[2] = {g0, g0 + kScanWarps};
+      const int nh = gi[1] < a.g ? 2 : 1;
+      const unsigned long long* const parts[2] = {a.part_keys + ((size_t)bi * a.g + gi[0]) * n_all,
+                                                  a.part_keys + ((size_t)bi * a.g + min(gi[1], a.g - 1)) * n_all};
+      stage(parts, nh, a.nsplit, KW);
+      unsigned long long r[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
+      for (int j = 0; j < nh; ++j) tournament(parts[j], win + (size_t)j * a.nsplit * KW, a.nsplit, KW, r[j][0], r[j][1]);
+      emit(gi, r);
+    }
+  } else {
+    // more ranges than one tournament takes: one head at a time; each group of kTour lists
+    // gives its best K, written back as list grp (a slot of group 0, already consumed), then
+    // a final tournament over the groups' lists
+    for (int g0 = warp; g0 < a.g; g0 += kScanWarps) {
+      unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + g0) * n_all;
+      unsigned long long r[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
       const int n_groups = (a.nsplit + kTour - 1) / kTour;
       for (int grp = 0; grp < n_groups; ++grp) {
-        tournament(parts + (size_t)grp * kTour * K, min(kTour, a.nsplit - grp * kTour), r0, r1);
+        const int nl = min(kTour, a.nsplit - grp * kTour);
+        const int KW = max(1, min(K, kStageKeys / nl));
+        const unsigned long long* const src[2] = {parts + (size_t)grp * kTour * K, parts};
+        stage(src, 1, nl, KW);
+        tournament(src[0], win, nl, KW, r[0][0], r[0][1]);
         __syncwarp();
-        if (lane < K) __stcg(parts + (size_t)grp * K + lane, r0);
-        if (lane + 32 < K) __stcg(parts + (size_t)grp * K + lane + 32, r1);
+        if (lane < K) __stcg(parts + (size_t)grp * K + lane, r[0][0]);
+        if (lane + 32 < K) __stcg(parts + (size_t)grp * K + lane + 32, r[0][1]);
         __threadfence_block();
         __syncwarp();
       }
-      tournament(parts, n_groups, r0, r1);
+      const int KW = max(1, min(K, kStageKeys / n_groups));
+      const unsigned long long* const src[2] = {parts, parts};
+      stage(src, 1, n_groups, KW);
+      tournament(parts, win, n_groups, KW, r[0][0], r[0][1]);
+      const int gi[2] = {g0, a.g};
+      emit(gi, r);
     }
-    emit(gi, r0, r1);
   }
   if constexpr (G > 1) {
     __syncthreads();  // the selection written above is read back below
@@ -405,7 +501,7 @@ __device__ __forceinline__ void load_row16(const T* src, float (&f)[16 / sizeof(
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kAttWarps * 32, 3) decode_attend_kernel(DecodeArgs a) {
   constexpr int CPL = D / 32;                  // output columns per lane (adjacent)
   constexpr int EPP = 16 / (int)sizeof(T);     // elements per 16-byte piece
   constexpr int PPR = D / EPP;                 // pieces per key row
@@ -544,51 +640,42 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
     if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
     return;
   }
-  // fusion weights, one warp per head.  The local branch's halves (2 NL of them) are
-  // combined into (mL, lL), LSE_local = mL + log lL; then lane s handles Top-K slot s
-  // (2 rounds cover K <= 64 slots), its chunk's (m, l) combined from its halves.
+  // fusion weights, one warp per head.  Every (m, l) pair and score the weights need is
+  // loaded at once, one L2 round trip: lane it < 2 NL holds local half it (NL <= 16), and
+  // lane s Top-K slots s and s + 32 (K <= 64) with both their halves.  The local halves
+  // give (mL, lL), LSE_local = mL + log lL; a slot's chunk takes its (m, l) from its halves.
   for (int hh = warp; hh < G; hh += kAttWarps) {
     const float* sc_row = a.ssel + ((size_t)bi * a.h + gi * G + hh) * K;
-    float mloc = -INFINITY, lloc = 0.f;
-    for (int it = lane; it < 2 * NL; it += 32) {
-      const float* pp = part + (size_t)it * part_stride + hh * (D + 2);
-      const float mh = __ldcg(pp);
-      if (mh == -INFINITY) continue;
-      const float lh = __ldcg(pp + 1);
-      const float nm = fmaxf(mloc, mh);
-      lloc = lloc * expf(mloc - nm) + lh * expf(mh - nm);
-      mloc = nm;
+    auto ml_of = [&](int it) {  // (m, l) of half item it; l is meaningful only where m is finite
+      return __ldcg(reinterpret_cast<const float2*>(part + (size_t)it * part_stride + hh * (D + 2)));
+    };
+    const float2 loc = lane < 2 * NL ? ml_of(lane) : make_float2(-INFINITY, 0.f);
+    float2 mlh[2][2];
+    float lg[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int sl = lane + 32 * rr;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) mlh[rr][h2] = sl < K ? ml_of(2 * (NL + sl) + h2) : make_float2(-INFINITY, 0.f);
+      lg[rr] = sl < K ? __ldcg(sc_row + sl) : -INFINITY;
     }
-    const float mL = warp_max(mloc);
-    const float lL = warp_sum(mloc == -INFINITY ? 0.f : lloc * expf(mloc - mL));
+    const float mL = warp_max(loc.x);
+    const float lL = warp_sum(loc.x == -INFINITY ? 0.f : loc.y * expf(loc.x - mL));
     const float lseL = mL + logf(lL);  // the own chunk always holds the new token: finite
-    float lg[2], ms[2], ls[2], mh[2][2];
+    float ms[2], ls[2];
     bool ok[2];
     float M = lseL;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int sl = lane + 32 * rr;
-      ok[rr] = false;
-      lg[rr] = -INFINITY;
-      ms[rr] = -INFINITY;
+      ms[rr] = fmaxf(mlh[rr][0].x, mlh[rr][1].x);
+      ok[rr] = ms[rr] != -INFINITY;
       ls[rr] = 0.f;
-      mh[rr][0] = mh[rr][1] = -INFINITY;
-      if (sl < K) {
-        float lh[2];
+      if (ok[rr]) {
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const float* pp = part + (size_t)(2 * (NL + sl) + h2) * part_stride + hh * (D + 2);
-          mh[rr][h2] = __ldcg(pp);
-          lh[h2] = mh[rr][h2] != -INFINITY ? __ldcg(pp + 1) : 0.f;
-        }
-        ms[rr] = fmaxf(mh[rr][0], mh[rr][1]);
-        ok[rr] = ms[rr] != -INFINITY;
-        if (ok[rr]) {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2)
-            if (mh[rr][h2] != -INFINITY) ls[rr] += lh[h2] * expf(mh[rr][h2] - ms[rr]);
-          lg[rr] = __ldcg(sc_row + sl);
-        }
+        for (int h2 = 0; h2 < 2; ++h2)
+          if (mlh[rr][h2].x != -INFINITY) ls[rr] += mlh[rr][h2].y * expf(mlh[rr][h2].x - ms[rr]);
+      } else {
+        lg[rr] = -INFINITY;
       }
       M = fmaxf(M, lg[rr]);
     }
@@ -598,10 +685,7 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
     for (int rr = 0; rr < 2; ++rr) z += ok[rr] ? expf(lg[rr] - M) : 0.f;
     const float Z = warp_sum(z) + expf(lseL - M);
     // local halves: exp(LSE_local - M)/Z * o/lL, i.e. exp(m_h - M)/Z * o_h per half
-    for (int it = lane; it < 2 * NL; it += 32) {
-      const float mhh = __ldcg(part + (size_t)it * part_stride + hh * (D + 2));
-      s_w[hh][it] = mhh == -INFINITY ? 0.f : expf(mhh - M) / Z;
-    }
+    if (lane < 2 * NL) s_w[hh][lane] = loc.x == -INFINITY ? 0.f : expf(loc.x - M) / Z;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int sl = lane + 32 * rr;
@@ -611,37 +695,53 @@ __global__ void __launch_bounds__(kAttWarps * 32) decode_attend_kernel(DecodeArg
         const float wsl = !ok[rr] ? 0.f : expf(lg[rr] - M) / (Z * ls[rr]);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
-          s_w[hh][2 * (NL + sl) + h2] = mh[rr][h2] == -INFINITY ? 0.f : wsl * expf(mh[rr][h2] - ms[rr]);
+          s_w[hh][2 * (NL + sl) + h2] = mlh[rr][h2].x == -INFINITY ? 0.f : wsl * expf(mlh[rr][h2].x - ms[rr]);
       }
     }
   }
   __syncthreads();
-  // weighted sum of the half-chunk outputs: thread = (head, column); the partials of a
-  // batch of items are all loaded before they are summed
-  constexpr int kFB = 16;
-  for (int x = t; x < G * D; x += blockDim.x) {
-    const int hh = x / D, col = x % D;
+  // weighted sum of the half-chunk outputs over items [i0, i1) for (head hh, column col);
+  // the partials of kFB items are all loaded before they are summed.  Absent halves were
+  // never written: their values are loaded but not used.
+  constexpr bool kSplit = 2 * G * D == kAttWarps * 32;  // see below
+  constexpr int kFB = kSplit ? 20 : 16;
+  auto wsum = [&](int hh, int col, int i0, int i1) {
     const float* pc = part + (size_t)hh * (D + 2) + 2 + col;
     float acc = 0.f;
-    for (int it0 = 0; it0 < n_items; it0 += kFB) {
-      float v[kFB], w[kFB];
+    for (int it0 = i0; it0 < i1; it0 += kFB) {
+      float v[kFB];
+#pragma unroll
+      for (int u = 0; u < kFB; ++u) v[u] = it0 + u < i1 ? __ldcg(pc + (size_t)(it0 + u) * part_stride) : 0.f;
 #pragma unroll
       for (int u = 0; u < kFB; ++u) {
-        const int it = it0 + u;
-        w[u] = it < n_items ? s_w[hh][it] : 0.f;
-        v[u] = w[u] != 0.f ? __ldcg(pc + (size_t)it * part_stride) : 0.f;  // absent halves were never written
+        const float w = it0 + u < i1 ? s_w[hh][it0 + u] : 0.f;
+        if (w != 0.f) acc = fmaf(v[u], w, acc);
       }
-#pragma unroll
-      for (int u = 0; u < kFB; ++u) acc = fmaf(v[u], w[u], acc);
     }
-    out[((size_t)bi * a.h + gi * G + hh) * D + col] = from_f<T>(acc);
+    return acc;
+  };
+  // With G D = 64 the CTA's 128 threads take (head, column) x (first or second half of
+  // the items), so that K + NL <= 20 costs one round trip; the halves meet in shared memory.
+  if constexpr (kSplit) {
+    __shared__ float s_acc[G * D];
+    const int x = t % (G * D), sp = t / (G * D);
+    const int n_half = (n_items + 1) / 2;
+    const float acc = wsum(x / D, x % D, sp * n_half, min(n_items, (sp + 1) * n_half));
+    if (sp == 1) s_acc[x] = acc;
+    __syncthreads();
+    if (sp == 0) out[((size_t)bi * a.h + gi * G) * D + x] = from_f<T>(acc + s_acc[x]);
+  } else {
+    for (int x = t; x < G * D; x += blockDim.x)
+      out[((size_t)bi * a.h + gi * G) * D + x] = from_f<T>(wsum(x / D, x % D, 0, n_items));
   }
   if (t == 0) a.att_ticket[(size_t)bi * a.g + gi] = 0;
 }
 
 template <typename T, int D, int G, typename S, int FPT, bool MULTI = false>
 static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)a.range * a.h * sizeof(float);  // scores
+  // the range's scores; afterwards, in the merging CTA, the warps' windows of list keys
+  const size_t smem = std::max((size_t)a.range * a.h * sizeof(float),
+                               (size_t)kScanWarps * kStageKeys * sizeof(unsigned long long));
   cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, S, FPT, MULTI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
