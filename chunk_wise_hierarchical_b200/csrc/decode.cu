@@ -15,6 +15,9 @@ int decode_splits(int batch, int max_chunks) {
   return max(lo, min(hi, want));
 }
 bool decode_supported(int h, int d) { return h * d <= 8 * kScanThreads * 4; }
+bool decode_merge_supported(int batch, int max_chunks, int top_k) {
+  return decode_merge_fits(decode_splits(batch, max_chunks), top_k);
+}
 
 #define HILS_DECLARE_SLICE(t, d, g) \
   cudaError_t run_decode_slice_##t##_##d##_##g(const DecodeArgs& a, cudaStream_t st);

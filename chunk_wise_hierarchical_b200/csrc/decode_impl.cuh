@@ -152,6 +152,115 @@ __device__ __forceinline__ void range_topk(const float* s_score, int H, int gi, 
   }
 }
 
+constexpr int kTour = 32 * kMaxListsPerLane;  // lists one tournament takes
+constexpr int kGroupKeys = 512;               // group results a grouped merge keeps (n_groups K)
+
+// Copies the first KW keys of each of n_lists lists of K keys (list l at parts + l K) into
+// the warp's window: list l, key p at win[l KW + p].  All loads are in flight at once.
+// Called by all 32 lanes.
+__device__ __forceinline__ void stage_lists(unsigned long long* win, const unsigned long long* parts, int n_lists,
+                                            int KW, int K) {
+  const int lane = threadIdx.x & 31;
+  const int n_win = n_lists * KW;
+  __syncwarp();  // the window's previous contents have been read
+  for (int x0 = 0; x0 < n_win; x0 += 32 * 16) {
+    unsigned long long tmp[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int x = x0 + 32 * u + lane;
+      tmp[u] = x < n_win ? __ldcg(parts + (size_t)(x / KW) * K + x % KW) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int x = x0 + 32 * u + lane;
+      if (x < n_win) win[x] = tmp[u];
+    }
+  }
+  __syncwarp();
+}
+
+// Tournament over n_lists <= kTour sorted lists of K keys (list l at parts + l K), whose
+// first KW keys are staged at w + l KW: each step is a warp max over the lists' heads (keys
+// are unique: they carry the chunk index), so a step waits on shared memory only; a list
+// that wins more than KW - 1 times reads on from global memory.  Lane l follows lists l,
+// l + 32, ..., holding each list's head and the key after it.  Returns the best K in
+// descending order: slot lane in r0, slot lane + 32 in r1 (0: empty).
+__device__ __forceinline__ void list_tournament(const unsigned long long* parts, const unsigned long long* w,
+                                                int n_lists, int KW, int K, unsigned long long& r0,
+                                                unsigned long long& r1) {
+  const int lane = threadIdx.x & 31;
+  auto key_at = [&](int l, int p) -> unsigned long long {
+    return p < KW ? w[l * KW + p] : p < K ? __ldcg(parts + (size_t)l * K + p) : 0ull;
+  };
+  int pos[kMaxListsPerLane];
+  unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
+#pragma unroll
+  for (int m = 0; m < kMaxListsPerLane; ++m) {
+    const int l = lane + 32 * m;
+    const bool live = l < n_lists;
+    pos[m] = 0;
+    head[m] = live ? key_at(l, 0) : 0ull;
+    next[m] = live ? key_at(l, 1) : 0ull;
+  }
+  r0 = 0ull;
+  r1 = 0ull;
+  for (int s = 0; s < K; ++s) {
+    unsigned long long lb = head[0];
+#pragma unroll
+    for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
+    const unsigned long long wb = warp_max_key(lb);
+    if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
+#pragma unroll
+    for (int m = 0; m < kMaxListsPerLane; ++m) {
+      if (head[m] == wb) {  // this lane's list m holds the winner: advance it
+        ++pos[m];
+        head[m] = next[m];
+        next[m] = key_at(lane + 32 * m, pos[m] + 1);
+      }
+    }
+    if ((s & 31) == lane) {
+      if (s < 32) r0 = wb;
+      else r1 = wb;
+    }
+  }
+}
+
+// Whether the merge of nsplit range lists of K keys fits: one tournament, or groups of
+// kTour lists whose results (n_groups K keys) stay in shared memory and are merged by one
+// more tournament (n_groups <= kTour).
+__host__ __device__ inline bool decode_merge_fits(int nsplit, int K) {
+  const int n_groups = (nsplit + kTour - 1) / kTour;
+  return nsplit <= kTour || (n_groups <= kTour && n_groups * K <= kGroupKeys);
+}
+
+// The Top-K of one KV head from its nsplit range lists (list l at parts + l K), by one warp:
+// one tournament, or with more than kTour lists a tournament per group of kTour lists
+// (results kept in grp_keys) and a final one over the groups' results.  win: the warp's
+// window of kStageKeys keys.  Returns slot lane in r0, slot lane + 32 in r1 (0: empty).
+__device__ __forceinline__ void merge_lists(const unsigned long long* parts, int nsplit, int K,
+                                            unsigned long long* win, unsigned long long* grp_keys,
+                                            unsigned long long& r0, unsigned long long& r1) {
+  const int lane = threadIdx.x & 31;
+  if (nsplit <= kTour) {
+    const int KW = max(1, min(K, kStageKeys / max(1, nsplit)));
+    stage_lists(win, parts, nsplit, KW, K);
+    list_tournament(parts, win, nsplit, KW, K, r0, r1);
+    return;
+  }
+  const int n_groups = (nsplit + kTour - 1) / kTour;
+  for (int grp = 0; grp < n_groups; ++grp) {
+    const int nl = min(kTour, nsplit - grp * kTour);
+    const int KW = max(1, min(K, kStageKeys / nl));
+    const unsigned long long* gp = parts + (size_t)grp * kTour * K;
+    stage_lists(win, gp, nl, KW, K);
+    list_tournament(gp, win, nl, KW, K, r0, r1);
+    if (lane < K) grp_keys[grp * K + lane] = r0;
+    if (lane + 32 < K) grp_keys[grp * K + lane + 32] = r1;
+  }
+  __syncwarp();
+  list_tournament(parts, grp_keys, n_groups, K, K, r0, r1);  // every key in shared memory
+}
+
 // Scan: CTA per (sequence, range of chunks), all heads.  A page's summaries of all
 // heads, [h][d] fp32, are one contiguous block; thread t holds float4 t + 256 k of it
 // (FPT per thread), so each page is read with fully coalesced 16-byte loads, PB pages
@@ -167,7 +276,6 @@ template <typename T, int D, int G, typename S, int FPT, bool MULTI>
 __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs a) {
   extern __shared__ __align__(16) float s_score[];  // [range][h]; reused by the merge
   __shared__ int s_page[kMaxRange];
-  __shared__ int s_last;
   constexpr int EPP = 16 / (int)sizeof(S);       // summary elements per 16-byte piece
   constexpr int QPR = D / EPP;                   // pieces per head row
   // load steps per batch: 8 pages' worth of fp32 pieces per thread (bf16 pieces hold twice
@@ -268,7 +376,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
   }
   __syncthreads();
 
-  // per KV head: this range's best K
+  // per KV head: this range's best K (merged into the head's Top-K by the attention kernel)
   const int E = nc <= 32 ? 1 : nc <= 64 ? 2 : nc <= 128 ? 4 : 8;
   for (int gi = warp; gi < a.g; gi += kScanWarps) {
     unsigned long long* part = a.part_keys + (((size_t)bi * a.g + gi) * a.nsplit + split) * K;
@@ -279,175 +387,6 @@ __global__ void __launch_bounds__(kScanThreads, 4) decode_scan_kernel(DecodeArgs
       default: range_topk<8, G>(s_score, H, gi, nc, c_lo, K, part); break;
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (t == 0) s_last = atomicAdd(a.scan_ticket + (size_t)bi * a.g, 1u) == (unsigned)(a.nsplit - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // ---- last CTA of the sequence: per KV head, merge the ranges' lists ----
-  // Every dependent round trip to L2 costs about as much here as the merge's arithmetic, so
-  // the merge is laid out to make few of them: the lists' leading keys are staged in shared
-  // memory with all loads in flight at once, a warp stages the lists of two heads together,
-  // and the block-table lookups of both heads' selections are issued together.
-  const int lane = t & 31;
-  const int n_all = a.nsplit * K;
-  unsigned long long* win = reinterpret_cast<unsigned long long*>(s_score) + (size_t)warp * kStageKeys;
-  // Copies the first KW keys of each of n_lists lists of nh heads (head j's lists at
-  // parts[j] + l K) into the window: head j, list l, key p at win[(j n_lists + l) KW + p].
-  auto stage = [&](const unsigned long long* const (&parts)[2], int nh, int n_lists, int KW) {
-    const int n_win = n_lists * KW, n_tot = nh * n_win;
-    __syncwarp();  // the window's previous contents have been read
-    for (int x0 = 0; x0 < n_tot; x0 += 32 * 16) {
-      unsigned long long tmp[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int x = x0 + 32 * u + lane;
-        const int j = x >= n_win, xx = x - j * n_win;
-        tmp[u] = x < n_tot ? __ldcg(parts[j] + (size_t)(xx / KW) * K + xx % KW) : 0ull;
-      }
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int x = x0 + 32 * u + lane;
-        if (x < n_tot) win[x] = tmp[u];
-      }
-    }
-    __syncwarp();
-  };
-  // Tournament over n_lists sorted lists of K keys (list l at parts + l K), whose first KW
-  // keys are staged at w + l KW: each step is a warp max over the lists' heads (keys are
-  // unique: they carry the chunk index), so a step waits on shared memory only; a list that
-  // wins more than KW - 1 times reads on from global memory.  Lane l follows lists l, l + 32,
-  // ..., holding each list's head and the key after it.  Returns the best K in descending
-  // order: slot lane in r0, slot lane + 32 in r1 (0: empty).
-  auto tournament = [&](const unsigned long long* parts, const unsigned long long* w, int n_lists, int KW,
-                        unsigned long long& r0, unsigned long long& r1) {
-    auto key_at = [&](int l, int p) -> unsigned long long {
-      return p < KW ? w[l * KW + p] : p < K ? __ldcg(parts + (size_t)l * K + p) : 0ull;
-    };
-    int pos[kMaxListsPerLane];
-    unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
-#pragma unroll
-    for (int m = 0; m < kMaxListsPerLane; ++m) {
-      const int l = lane + 32 * m;
-      const bool live = l < n_lists;
-      pos[m] = 0;
-      head[m] = live ? key_at(l, 0) : 0ull;
-      next[m] = live ? key_at(l, 1) : 0ull;
-    }
-    r0 = 0ull;
-    r1 = 0ull;
-    for (int s = 0; s < K; ++s) {
-      unsigned long long lb = head[0];
-#pragma unroll
-      for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
-      const unsigned long long wb = warp_max_key(lb);
-      if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
-#pragma unroll
-      for (int m = 0; m < kMaxListsPerLane; ++m) {
-        if (head[m] == wb) {  // this lane's list m holds the winner: advance it
-          ++pos[m];
-          head[m] = next[m];
-          next[m] = key_at(lane + 32 * m, pos[m] + 1);
-        }
-      }
-      if ((s & 31) == lane) {
-        if (s < 32) r0 = wb;
-        else r1 = wb;
-      }
-    }
-  };
-  // Writes the selections of heads gi[0] and gi[1] (gi >= g: none): keys r[j][0] for slot
-  // lane and r[j][1] for slot lane + 32, in descending order (0: empty).  The four block-table
-  // reads are issued before any is used.
-  auto emit = [&](const int (&gi)[2], const unsigned long long (&r)[2][2]) {
-    int c[2][2], pg[2][2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const bool live = gi[j] < a.g && lane + 32 * q < K;
-        c[j][q] = live && r[j][q] ? (int)key_chunk(r[j][q]) : -1;
-        pg[j][q] = c[j][q] >= 0 ? bt[c[j][q]] : -1;
-      }
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int sl = lane + 32 * q;
-        if (gi[j] >= a.g || sl >= K) continue;
-        a.idx[((size_t)bi * a.g + gi[j]) * K + sl] = c[j][q];
-        a.sel_page[((size_t)bi * a.g + gi[j]) * K + sl] = pg[j][q];
-        // G = 1: the selection key is the head's own score
-        if (G == 1)
-          a.ssel[((size_t)bi * a.h + gi[j]) * K + sl] = r[j][q] ? unorderable((uint32_t)(r[j][q] >> 32)) : -INFINITY;
-      }
-  };
-  constexpr int kTour = 32 * kMaxListsPerLane;  // lists one tournament takes
-  if (a.nsplit <= kTour) {
-    // heads in pairs (warp, warp + kScanWarps), then (warp + 2 kScanWarps, ...), ...: each
-    // head's lists get half the window
-    const int KW = max(1, min(K, (kStageKeys / 2) / a.nsplit));
-    for (int g0 = warp; g0 < a.g; g0 += 2 * kScanWarps) {
-      const int gi[2] = {g0, g0 + kScanWarps};
-      const int nh = gi[1] < a.g ? 2 : 1;
-      const unsigned long long* const parts[2] = {a.part_keys + ((size_t)bi * a.g + gi[0]) * n_all,
-                                                  a.part_keys + ((size_t)bi * a.g + min(gi[1], a.g - 1)) * n_all};
-      stage(parts, nh, a.nsplit, KW);
-      unsigned long long r[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
-      for (int j = 0; j < nh; ++j) tournament(parts[j], win + (size_t)j * a.nsplit * KW, a.nsplit, KW, r[j][0], r[j][1]);
-      emit(gi, r);
-    }
-  } else {
-    // more ranges than one tournament takes: one head at a time; each group of kTour lists
-    // gives its best K, written back as list grp (a slot of group 0, already consumed), then
-    // a final tournament over the groups' lists
-    for (int g0 = warp; g0 < a.g; g0 += kScanWarps) {
-      unsigned long long* parts = a.part_keys + ((size_t)bi * a.g + g0) * n_all;
-      unsigned long long r[2][2] = {{0ull, 0ull}, {0ull, 0ull}};
-      const int n_groups = (a.nsplit + kTour - 1) / kTour;
-      for (int grp = 0; grp < n_groups; ++grp) {
-        const int nl = min(kTour, a.nsplit - grp * kTour);
-        const int KW = max(1, min(K, kStageKeys / nl));
-        const unsigned long long* const src[2] = {parts + (size_t)grp * kTour * K, parts};
-        stage(src, 1, nl, KW);
-        tournament(src[0], win, nl, KW, r[0][0], r[0][1]);
-        __syncwarp();
-        if (lane < K) __stcg(parts + (size_t)grp * K + lane, r[0][0]);
-        if (lane + 32 < K) __stcg(parts + (size_t)grp * K + lane + 32, r[0][1]);
-        __threadfence_block();
-        __syncwarp();
-      }
-      const int KW = max(1, min(K, kStageKeys / n_groups));
-      const unsigned long long* const src[2] = {parts, parts};
-      stage(src, 1, n_groups, KW);
-      tournament(parts, win, n_groups, KW, r[0][0], r[0][1]);
-      const int gi[2] = {g0, a.g};
-      emit(gi, r);
-    }
-  }
-  if constexpr (G > 1) {
-    __syncthreads();  // the selection written above is read back below
-    // each head's own score of the selected chunks: one warp per (KV head, slot, head)
-    for (int x = warp; x < a.g * K * G; x += kScanWarps) {
-      const int gi = x / (K * G), s = (x / G) % K, hh = x % G;
-      const int c = a.idx[((size_t)bi * a.g + gi) * K + s];
-      float sc = -INFINITY;
-      if (c >= 0) {
-        const int p = bt[c];
-        const S* kb = static_cast<const S*>(a.kbar_pages) + ((size_t)p * H + gi * G + hh) * D;
-        const T* qr = static_cast<const T*>(a.q) + ((size_t)bi * H + gi * G + hh) * D;
-        float acc = 0.f;
-#pragma unroll
-        for (int e = lane; e < D; e += 32) acc = fmaf(to_f(qr[e]), to_f(kb[e]), acc);
-        acc = warp_sum(acc);
-        sc = fmaf(acc, a.scale, __ldg(a.hbias_pages + (size_t)p * H + gi * G + hh));
-      }
-      if (lane == 0) a.ssel[((size_t)bi * H + gi * G + hh) * K + s] = sc;
-    }
-  }
-  if (t == 0) a.scan_ticket[(size_t)bi * a.g] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -501,12 +440,15 @@ __device__ __forceinline__ void load_row16(const T* src, float (&f)[16 / sizeof(
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kAttWarps * 32, 3) decode_attend_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kAttWarps * 32, G == 1 ? 8 : 3) decode_attend_kernel(DecodeArgs a) {
   constexpr int CPL = D / 32;                  // output columns per lane (adjacent)
   constexpr int EPP = 16 / (int)sizeof(T);     // elements per 16-byte piece
   constexpr int PPR = D / EPP;                 // pieces per key row
   __shared__ __align__(16) float qS[G][D];
   __shared__ float s_w[G][2 * (kMaxTopK + kMaxDecodeLocal)];  // fusion weight of each half chunk, per head
+  __shared__ __align__(16) unsigned long long s_win[kStageKeys];  // the merging warp's window of list keys
+  __shared__ unsigned long long s_grp[kGroupKeys];                // group results of a grouped merge
+  __shared__ unsigned long long s_key[kMaxTopK];                  // the selection: key of each slot (0: empty)
   __shared__ int s_last;
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -623,9 +565,59 @@ __global__ void __launch_bounds__(kAttWarps * 32, 3) decode_attend_kernel(Decode
              c == own ? L - own * kChunk : kChunk);
   }
   pdl_wait_primary();
-  if (item >= 2 * NL && item < n_items && L > 0) {
-    const size_t slot = ((size_t)bi * a.g + gi) * K + (item >> 1) - NL;
-    run_item(a.idx[slot], a.sel_page[slot], kChunk);
+  // The Top-K of this KV head, merged from the scan's range lists by warp 0 of every CTA of
+  // the (sequence, KV head): the scan grid has completed, so no CTA waits on another.
+  if (K > 0) {
+    if (warp == 0) {
+      unsigned long long r0, r1;
+      merge_lists(a.part_keys + ((size_t)bi * a.g + gi) * a.nsplit * K, a.nsplit, K, s_win, s_grp, r0, r1);
+      if (lane < K) s_key[lane] = r0;
+      if (lane + 32 < K) s_key[lane + 32] = r1;
+    }
+    __syncthreads();
+  }
+  if (item >= 2 * NL && item < n_items) {
+    const int sl = (item >> 1) - NL;
+    const unsigned long long key = s_key[sl];
+    const int c = key ? (int)key_chunk(key) : -1;  // a candidate: c < max_chunks
+    const int p = c >= 0 ? a.block_table[(size_t)bi * a.max_chunks + c] : -1;
+    if (L > 0) run_item(c, p, kChunk);
+    if (hf == 0) {
+      // the slot's outputs, written once: its chunk, and each query head's own score of it
+      // (G = 1: the selection key is the head's own score)
+      if (lane == 0) a.idx[((size_t)bi * a.g + gi) * K + sl] = c;
+      if constexpr (G == 1) {
+        if (lane == 0) a.ssel[((size_t)bi * a.h + gi) * K + sl] = key ? unorderable((uint32_t)(key >> 32)) : -INFINITY;
+      } else {
+        float acc[G];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) acc[hh] = 0.f;
+        if (c >= 0 && p >= 0 && p < a.n_pages) {  // a selected chunk's page was valid when it was scored
+          const size_t row0 = ((size_t)p * a.h + gi * G) * D;
+          if (a.kbar_bf16) {
+            const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.kbar_pages) + row0;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+              for (int e = lane; e < D; e += 32) acc[hh] = fmaf(qS[hh][e], __bfloat162float(kb[hh * D + e]), acc[hh]);
+          } else {
+            const float* kb = static_cast<const float*>(a.kbar_pages) + row0;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+              for (int e = lane; e < D; e += 32) acc[hh] = fmaf(qS[hh][e], __ldg(kb + hh * D + e), acc[hh]);
+          }
+        }
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float dot = warp_sum(acc[hh]);
+          const float sc = c >= 0 && p >= 0 && p < a.n_pages
+                               ? fmaf(dot, a.scale, __ldg(a.hbias_pages + (size_t)p * a.h + gi * G + hh))
+                               : -INFINITY;
+          if (lane == 0) a.ssel[((size_t)bi * a.h + gi * G + hh) * K + sl] = sc;
+        }
+      }
+    }
   }
 
   __threadfence();
@@ -739,9 +731,7 @@ __global__ void __launch_bounds__(kAttWarps * 32, 3) decode_attend_kernel(Decode
 
 template <typename T, int D, int G, typename S, int FPT, bool MULTI = false>
 static cudaError_t launch_scan(const DecodeArgs& a, cudaStream_t st) {
-  // the range's scores; afterwards, in the merging CTA, the warps' windows of list keys
-  const size_t smem = std::max((size_t)a.range * a.h * sizeof(float),
-                               (size_t)kScanWarps * kStageKeys * sizeof(unsigned long long));
+  const size_t smem = (size_t)a.range * a.h * sizeof(float);  // the range's scores
   cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, D, G, S, FPT, MULTI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

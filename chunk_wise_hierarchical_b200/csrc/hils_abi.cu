@@ -426,6 +426,7 @@ hils_status hils_decode_ex(const hils_shape* s, const void* q, const void* k_pag
   if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) > kMaxDecodeLocal) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
+  if (!hils::decode_merge_supported(s->batch, max_chunks, s->top_k)) return HILS_ERR_UNSUPPORTED;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
     return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(kbar_pages) ||
@@ -551,6 +552,7 @@ hils_status hils_decode_static(const hils_shape* s, const void* q, const void* k
   if (!hils::decode_supported(s->heads_q, s->head_dim) || n_local(s) > kMaxDecodeLocal) return HILS_ERR_UNSUPPORTED;
   if (max_chunks <= 0 || n_pages <= 0) return HILS_ERR_INVALID_ARG;
   if ((long long)max_chunks > ((long long)s->seq_len + s->chunk - 1) / s->chunk) return HILS_ERR_INVALID_ARG;
+  if (!hils::decode_merge_supported(s->batch, max_chunks, s->top_k)) return HILS_ERR_UNSUPPORTED;
   if (!q || !k_pages || !v_pages || !kbar_pages || !hbias_pages || !block_table || !seq_lens || !out)
     return HILS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(kbar_pages) ||

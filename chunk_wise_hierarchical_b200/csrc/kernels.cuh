@@ -74,11 +74,11 @@ struct DecodeArgs {
   const int32_t* seq_lens;     // [b]
   void* out;                   // [b,h,d]
   int32_t* idx;                // [b,g,K]
-  int32_t* sel_page;           // [b,g,K] page of each selected chunk
+  int32_t* sel_page;           // [b,g,K] reserved (the attention kernel looks pages up itself)
   float* ssel;                 // [b,h,K]
   unsigned long long* part_keys;  // [b,g,nsplit,K] per-range Top-K lists
   float* part_att;             // [b,g,2(K+n_local),G,d+2]: per half chunk (max, sum, unnormalised output)
-  unsigned* scan_ticket;       // [b,g] (the scan uses entry (b, 0))
+  unsigned* scan_ticket;       // [b,g] reserved (the scan takes no ticket)
   unsigned* att_ticket;        // [b,g]
   unsigned* err;
   bool kbar_bf16;              // compact summary cache (bf16 models only)
@@ -90,6 +90,8 @@ struct DecodeArgs {
 };
 int decode_splits(int batch, int max_chunks);
 bool decode_supported(int h, int d);  // the scan holds a page's summaries of all heads: h * d <= 8192
+// whether the Top-K merge of the scan's range lists fits the attention kernel's shared memory
+bool decode_merge_supported(int batch, int max_chunks, int top_k);
 cudaError_t run_decode(DecodeArgs a, cudaStream_t st);
 
 // Row-wise attention + fusion (one warp per query and KV group).
