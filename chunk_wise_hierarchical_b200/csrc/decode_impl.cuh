@@ -184,18 +184,20 @@ __device__ __forceinline__ void stage_lists(unsigned long long* win, const unsig
 // are unique: they carry the chunk index), so a step waits on shared memory only; a list
 // that wins more than KW - 1 times reads on from global memory.  Lane l follows lists l,
 // l + 32, ..., holding each list's head and the key after it.  Returns the best K in
-// descending order: slot lane in r0, slot lane + 32 in r1 (0: empty).
-__device__ __forceinline__ void list_tournament(const unsigned long long* parts, const unsigned long long* w,
-                                                int n_lists, int KW, int K, unsigned long long& r0,
-                                                unsigned long long& r1) {
+// descending order: slot lane in r0, slot lane + 32 in r1 (0: empty).  LPL: lists per lane
+// (n_lists <= 32 LPL).
+template <int LPL>
+__device__ __forceinline__ void list_tournament_n(const unsigned long long* parts, const unsigned long long* w,
+                                                  int n_lists, int KW, int K, unsigned long long& r0,
+                                                  unsigned long long& r1) {
   const int lane = threadIdx.x & 31;
   auto key_at = [&](int l, int p) -> unsigned long long {
     return p < KW ? w[l * KW + p] : p < K ? __ldcg(parts + (size_t)l * K + p) : 0ull;
   };
-  int pos[kMaxListsPerLane];
-  unsigned long long head[kMaxListsPerLane], next[kMaxListsPerLane];
+  int pos[LPL];
+  unsigned long long head[LPL], next[LPL];
 #pragma unroll
-  for (int m = 0; m < kMaxListsPerLane; ++m) {
+  for (int m = 0; m < LPL; ++m) {
     const int l = lane + 32 * m;
     const bool live = l < n_lists;
     pos[m] = 0;
@@ -207,11 +209,11 @@ __device__ __forceinline__ void list_tournament(const unsigned long long* parts,
   for (int s = 0; s < K; ++s) {
     unsigned long long lb = head[0];
 #pragma unroll
-    for (int m = 1; m < kMaxListsPerLane; ++m) lb = head[m] > lb ? head[m] : lb;
+    for (int m = 1; m < LPL; ++m) lb = head[m] > lb ? head[m] : lb;
     const unsigned long long wb = warp_max_key(lb);
     if (wb == 0ull) break;  // every list is exhausted (warp-uniform)
 #pragma unroll
-    for (int m = 0; m < kMaxListsPerLane; ++m) {
+    for (int m = 0; m < LPL; ++m) {
       if (head[m] == wb) {  // this lane's list m holds the winner: advance it
         ++pos[m];
         head[m] = next[m];
@@ -223,6 +225,14 @@ __device__ __forceinline__ void list_tournament(const unsigned long long* parts,
       else r1 = wb;
     }
   }
+}
+
+__device__ __forceinline__ void list_tournament(const unsigned long long* parts, const unsigned long long* w,
+                                                int n_lists, int KW, int K, unsigned long long& r0,
+                                                unsigned long long& r1) {
+  if (n_lists <= 32) list_tournament_n<1>(parts, w, n_lists, KW, K, r0, r1);
+  else if (n_lists <= 64) list_tournament_n<2>(parts, w, n_lists, KW, K, r0, r1);
+  else list_tournament_n<kMaxListsPerLane>(parts, w, n_lists, KW, K, r0, r1);
 }
 
 // Whether the merge of nsplit range lists of K keys fits: one tournament, or groups of

@@ -293,6 +293,9 @@ HILS_API hils_status hils_backward(const hils_shape* shape, const void* q, const
  *   topk_idx_out [batch, heads_kv, top_k] int32 or NULL
  *   ws           workspace of hils_workspace_size(HILS_OP_DECODE) bytes
  * Page ids outside [0, n_pages) are skipped and flagged in the error word.
+ * max_chunks is limited to about 2^24 / top_k (the Top-K merge of the
+ * scan's per-range lists runs in shared memory); beyond it the call returns
+ * HILS_ERR_UNSUPPORTED.
  */
 HILS_API hils_status hils_decode(const hils_shape* shape, const void* q, const void* k_pages,
                         const void* v_pages, const float* kbar_pages, const float* hbias_pages,
@@ -324,12 +327,15 @@ HILS_API hils_status hils_decode(const hils_shape* shape, const void* q, const v
  * Every call on a device uses the same array: calls whose kernels may run at
  * the same time (different streams with no ordering between them, or
  * different host threads) race on it and corrupt each other's results; order
- * them on one stream or with events.  Its ticket counters must start at zero:
- * they are zero when the library's device code is loaded, and each call that
- * completes leaves them at zero again.  A call that returns HILS_ERR_CUDA
- * after its first kernel was enqueued (the second launch failed) can leave
- * tickets non-zero; later calls on that device then return wrong results
- * until the library's device code is loaded again (a new process).
+ * them on one stream or with events.  Its ticket counters (taken by the
+ * attention kernel's CTAs, the last of each (sequence, KV head) resetting
+ * its own) must start at zero: they are zero when the library's device code
+ * is loaded, and each call whose attention kernel runs to completion leaves
+ * them at zero again.  A call whose second launch fails (HILS_ERR_CUDA after
+ * the first kernel was enqueued) touches no ticket; an attention kernel that
+ * starts but does not complete can leave tickets non-zero, and later calls
+ * on that device then return wrong results until the library's device code
+ * is loaded again (a new process).
  * kbar_pages must be the fp32 summary cache (this entry point has no
  * summary_dtype argument).
  */
