@@ -5,22 +5,21 @@
 // 1. decode_scan_kernel -- grid (sequence, range of candidate chunks).  Each CTA
 //    reads the cached summaries of its range page by page, all heads at once (a
 //    page's [h][d] fp32 block is contiguous), scores them (q . kbar * scale + H, GQA
-//    max over the group's heads) and, one warp per KV head, sorts the range's keys
-//    and writes its best K.  The last CTA of the sequence -- an atomic ticket; no
-//    CTA waits on another -- merges the ranges' lists into the final Top-K and
-//    writes each head's own score of the selected chunks.
-// 2. decode_attend_kernel -- one warp per chunk (own chunk or one Top-K slot),
-//    all G heads sharing each K/V load, K and V staged in shared memory with
-//    cp.async.  The own chunk does not depend on the selection and is
-//    computed before the kernel waits for the scan grid.  Each warp writes
-//    its chunk's (max, sum, unnormalised output); the last CTA of the
-//    (sequence, KV head) fuses them with the inter-chunk softmax of notes
-//    section 5.3 (own chunk at its exact log-mass).
-// Tickets are reset by the CTA that consumes them, so both kernels can be
-// replayed (CUDA graphs) without clearing the workspace.
+//    max over the group's heads) and, one warp per KV head, writes the range's best
+//    K keys as a sorted list.
+// 2. decode_attend_kernel -- one warp per half chunk (32 keys) of the local
+//    branch or of one Top-K slot, all G heads sharing each K/V load.  The local
+//    branch does not depend on the selection and is computed before the kernel
+//    waits for the scan grid.  Then warp 0 of every CTA merges its KV head's range
+//    lists into the Top-K (a warp tournament over the sorted lists, staged in
+//    shared memory), and each slot's warps look up the chunk's page and attend to
+//    it.  Each warp writes its half's (max, sum, unnormalised output); the last CTA
+//    of the (sequence, KV head) -- an atomic ticket; no CTA waits on another --
+//    fuses them with the inter-chunk softmax of notes section 5.3 (local branch at
+//    its exact log-mass).
+// The ticket is reset by the CTA that consumes it, so both kernels can be replayed
+// (CUDA graphs) without clearing the workspace.
 #pragma once
-#include <algorithm>
-
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -276,8 +275,8 @@ __device__ __forceinline__ void merge_lists(const unsigned long long* parts, int
 // (FPT per thread), so each page is read with fully coalesced 16-byte loads, PB pages
 // in flight per thread.  Per (chunk, head) the dot with q is reduced over the d/4
 // lanes of the head row, scaled and biased by H into shared memory; then one warp per
-// KV head sorts the range's keys and writes its best K.  The last CTA of the sequence
-// (atomic ticket; no CTA waits on another) merges the ranges' lists.
+// KV head takes the range's best K and writes them as a sorted list, which the attention
+// kernel merges with the other ranges' lists.
 // Four CTAs per SM (64 registers a thread): a page gather's bandwidth grows with the
 // warps resident on the SM far more than with the loads each warp has in flight.
 // S: element type of the cached summaries (fp32, or bf16 for the compact cache).

@@ -146,6 +146,27 @@ def test_decode_window_beyond_the_decode_limit_is_unsupported():
                            fake, 1 << 30, None) == 2
 
 
+def test_decode_beyond_the_merge_limit_is_unsupported():
+    """The attention kernel merges the scan's per-range Top-K lists in shared memory:
+    more than 128 ranges are merged in groups of 128 whose results (groups x top_k keys)
+    must fit 512 keys.  With one sequence and top_k = 64 that allows 8 groups, i.e.
+    1024 ranges of 256 chunks: max_chunks = 2^18 passes this check, 2^18 + 256 does not.
+    Both hils_decode and hils_decode_static refuse it before any launch."""
+    lib = hils.lib()
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the call fails validation first
+    mc = (1 << 18) + 256
+    s = _shape(batch=1, heads_q=8, heads_kv=8, top_k=64, seq_len=mc * 64)
+    assert lib.hils_decode(ctypes.byref(s), fake, fake, fake, fake, fake, fake, mc, fake, 4, fake, None,
+                           fake, 1 << 40, None) == 2
+    assert lib.hils_decode_static(ctypes.byref(s), fake, fake, fake, fake, fake, fake, mc, fake, 4, fake,
+                                  None, None, None) == 2
+    # top_k = 16 allows 32 groups: the same cache is within the limit (the call then fails
+    # later, for lack of a workspace, not as unsupported)
+    s16 = _shape(batch=1, heads_q=8, heads_kv=8, top_k=16, seq_len=mc * 64)
+    assert lib.hils_decode(ctypes.byref(s16), fake, fake, fake, fake, fake, fake, mc, fake, 4, fake, None,
+                           fake, 0, None) == 3
+
+
 def test_decode_static_binding_rejects_a_bf16_summary_cache():
     """hils_decode_static reads fp32 summaries only: the binding refuses a bf16
     cache before any pointer reaches the library."""
