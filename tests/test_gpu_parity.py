@@ -315,6 +315,16 @@ def test_decode_sliding_window_local_branch(dtype, window, G):
     _check_decode(di, out, idx, 3, [(b, g) for b in range(6) for g in range(2)], window=window)
 
 
+@pytest.mark.parametrize("G", [1, 4])
+def test_decode_top_k_above_32(G):
+    """Top-K slots 32 .. K-1 (the second key register of the range lists and of the merge),
+    K = 40, with sequences of 48 and 70 candidate chunks and one shorter than K."""
+    di = decode_inputs(3, 2 * G, 2, 0, 64, top_k=40, dtype="bf16", seed=9,
+                       seq_lens=[64 * 49 + 5, 64 * 71, 64 * 20 + 1], spare_pages=2)
+    out, idx = _gpu_decode(di, 40)
+    _check_decode(di, out, idx, 40, [(b, g) for b in range(3) for g in range(2)])
+
+
 def test_decode_gqa_d128():
     di = decode_inputs(2, 8, 1, 0, 128, top_k=6, dtype="bf16", seed=5, seq_lens=[900, 2000])
     out, idx = _gpu_decode(di, 6)
