@@ -122,6 +122,61 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _expect(t, shape, dtypes, name):
+    """Raises unless tensor t has exactly this shape and one of these dtypes: the kernels
+    read every tensor at the extent the shape implies."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {list(shape)}, got {list(t.shape)}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+
+
+def _same_device(ref, *ts):
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError("every tensor must be on q's device")
+
+
+def check_prefill_args(shape, q, k, v, landmark, out=None):
+    """The prefill inputs against the shape: q [b,h,N,d]; k, v [b,g,N,d] and landmark
+    [b,h,N//64,d] in q's dtype; out (if given) like q."""
+    s = shape
+    _expect(q, (s.batch, s.heads_q, s.seq_len, s.head_dim), (torch.bfloat16, torch.float32), "q")
+    if _dt(q) != s.dtype:
+        raise TypeError("q's dtype does not match the prepared shape")
+    kv = (s.batch, s.heads_kv, s.seq_len, s.head_dim)
+    _expect(k, kv, (q.dtype,), "k")
+    _expect(v, kv, (q.dtype,), "v")
+    if landmark is not None:
+        _expect(landmark, (s.batch, s.heads_q, s.seq_len // s.chunk, s.head_dim), (q.dtype,), "landmark")
+    if out is not None:
+        _expect(out, q.shape, (q.dtype,), "out")
+    _same_device(q, k, v, landmark, out)
+
+
+def check_decode_args(shape, q, k_pages, v_pages, kbar_pages, hbias_pages, seq_lens, out=None, topk_idx=None):
+    """The decode inputs against the shape: q [b,h,d]; k/v pages [P,g,64,d] in q's dtype;
+    kbar pages [P,h,d] fp32 (or bf16, the compact cache); hbias pages [P,h] fp32; seq_lens
+    [b] int32; topk_idx (if given) int32 with at least b*g*K entries; out (if given) like q."""
+    s = shape
+    _expect(q, (s.batch, s.heads_q, s.head_dim), (torch.bfloat16, torch.float32), "q")
+    if _dt(q) != s.dtype:
+        raise TypeError("q's dtype does not match the prepared shape")
+    P = k_pages.shape[0] if k_pages.dim() == 4 else -1
+    _expect(k_pages, (P, s.heads_kv, s.chunk, s.head_dim), (q.dtype,), "k_pages")
+    _expect(v_pages, (P, s.heads_kv, s.chunk, s.head_dim), (q.dtype,), "v_pages")
+    _expect(kbar_pages, (P, s.heads_q, s.head_dim), (torch.float32, torch.bfloat16), "kbar_pages")
+    _expect(hbias_pages, (P, s.heads_q), (torch.float32,), "hbias_pages")
+    _expect(seq_lens, (s.batch,), (torch.int32,), "seq_lens")
+    if topk_idx is not None and (topk_idx.dtype != torch.int32 or topk_idx.numel() < s.batch * s.heads_kv * s.top_k):
+        raise TypeError("topk_idx must be an int32 tensor of at least batch * heads_kv * top_k entries")
+    if out is not None:
+        _expect(out, q.shape, (q.dtype,), "out")
+    _same_device(q, k_pages, v_pages, kbar_pages, hbias_pages, seq_lens, out, topk_idx)
+
+
 def _check(st: int, where: str):
     if st != 0:
         raise HilsError(st, where)
@@ -166,6 +221,10 @@ def summarize_paged(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages, 
     h = landmark_pages.shape[1]
     if page_ids.dtype != torch.int32:
         raise TypeError("page_ids must be int32")
+    _expect(landmark_pages, (n_pages, h, d), (k_pages.dtype,), "landmark_pages")
+    _expect(kbar_pages, (n_pages, h, d), (torch.float32, torch.bfloat16), "kbar_pages")
+    _expect(hbias_pages, (n_pages, h), (torch.float32,), "hbias_pages")
+    _same_device(k_pages, landmark_pages, page_ids, kbar_pages, hbias_pages)
     sh = make_shape(0, h, g, d, 0, 0, _dt(k_pages), chunk=chunk, scale=scale or 0.0)
     _check(lib().hils_summarize_paged_ex(ctypes.byref(sh), _ptr(k_pages), _ptr(landmark_pages), _ptr(page_ids),
                                          int(page_ids.numel()), int(n_pages), _ptr(kbar_pages), _dt(kbar_pages),
@@ -177,6 +236,9 @@ def select(q, kbar, hbias, top_k, heads_kv, scale=None, stream=None, with_scores
     given, is the workspace whose error word the kernels report into."""
     b, h, n, d = q.shape
     sh = make_shape(b, h, heads_kv, d, n, top_k, _dt(q), scale=scale or 0.0, window=window)
+    _expect(kbar, (b, h, n // 64, d), (torch.float32,), "kbar")
+    _expect(hbias, (b, h, n // 64), (torch.float32,), "hbias")
+    _same_device(q, kbar, hbias, ws)
     idx = torch.empty((b, heads_kv, n, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, h, n, top_k), dtype=torch.float32, device=q.device) if with_scores else None
     if ws is None:
@@ -198,11 +260,8 @@ class Prefill:
 
     def __call__(self, q, k, v, landmark, out=None, topk_idx=None, stream=None, lse=None):
         s = self.shape
-        if q.shape != (s.batch, s.heads_q, s.seq_len, s.head_dim) or _dt(q) != s.dtype:
-            raise ValueError("q does not match the prepared shape")
-        for t in (k, v, landmark):
-            if t.dtype != q.dtype:
-                raise TypeError("q, k, v and landmark must share a dtype")
+        check_prefill_args(s, q, k, v, landmark, out)
+        _same_device(q, lse, topk_idx, self.ws)
         if out is None:
             out = torch.empty_like(q)
         if lse is not None and (lse.dtype != torch.float32 or lse.shape != q.shape[:3]):
@@ -258,6 +317,8 @@ def attend_selected(q, k, v, topk_idx, topk_score, scale=None, out=None, ws=None
         raise ValueError("topk_idx must be [b, heads_kv, N, K] and topk_score [b, heads_q, N, K]")
     if lse is not None and (lse.dtype != torch.float32 or lse.shape != (b, h, n)):
         raise ValueError("lse must be fp32 [b, h, N]")
+    check_prefill_args(sh, q, k, v, None, out)
+    _same_device(q, topk_idx, topk_score, lse, ws)
     if out is None:
         out = torch.empty_like(q)
     if ws is None:
@@ -287,6 +348,8 @@ class Decode:
             raise TypeError("block_table and seq_lens must be int32")
         if block_table.shape != (s.batch, self.max_chunks):
             raise ValueError("block_table must be [batch, max_chunks]")
+        check_decode_args(s, q, k_pages, v_pages, kbar_pages, hbias_pages, seq_lens, out, topk_idx)
+        _same_device(q, block_table, self.ws)
         if out is None:
             out = torch.empty_like(q)
         _check(lib().hils_decode_ex(ctypes.byref(s), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kbar_pages),
@@ -365,6 +428,8 @@ def backward(q, k, v, landmark, out, lse, topk_idx, topk_score, dout, scale=None
     if topk_score.dtype != torch.float32 or topk_score.shape != (b, h, n, K):
         raise ValueError("topk_score must be fp32 [b, heads_q, N, K]")
     sh = make_shape(b, h, g, d, n, K, HILS_BF16, scale=scale or 0.0, window=window)
+    check_prefill_args(sh, q, k, v, landmark, out)
+    _same_device(q, lse, topk_idx, topk_score, dout, ws)
     f32 = dict(dtype=torch.float32, device=q.device)
     dq = torch.empty((b, h, n, d), **f32)
     dk = torch.empty((b, g, n, d), **f32)

@@ -39,7 +39,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_replicas_take_the_max_time():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this (threaded) process
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     assert sorted(out.keys()) == [0, 1]
     for r in range(world):
